@@ -1,0 +1,172 @@
+"""fp64 CPU oracle for the DBF layer forward (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its
+``cpu_baseline`` and ``--impl reference`` legs) may import this package.  The
+product path in ``binary_factorized_weight_b200`` never imports it, and this
+package never imports the product: the two share no code.  The arithmetic lives
+in ``dbf_oracle.c`` (plain C loops, fp64); this module only marshals numpy
+arrays into it.
+
+Each function cites the passage of "Addition is almost all you need:
+Compressing large language models with double binary factorization" it
+follows (gist.science technical summary, section 2.1, and sciencestack.ai
+Figure 1).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _setup(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    i64, dbl, vp = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_words_per_row.argtypes = [i64]
+    lib.oracle_words_per_row.restype = i64
+    lib.oracle_unpack_signs.argtypes = [vp, i64, i64, vp]
+    lib.oracle_unpack_signs.restype = i64
+    lib.oracle_pack_signs.argtypes = [vp, i64, i64, vp]
+    lib.oracle_pack_signs.restype = None
+    lib.oracle_forward_staged.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, vp]
+    lib.oracle_forward_staged.restype = None
+    lib.oracle_dense_weight.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
+    lib.oracle_dense_weight.restype = None
+    lib.oracle_forward_dense.argtypes = [vp, vp, i64, i64, i64, vp]
+    lib.oracle_forward_dense.restype = None
+    lib.oracle_bits_per_weight.argtypes = [i64, i64, i64]
+    lib.oracle_bits_per_weight.restype = dbl
+    lib.oracle_scale_bits_per_weight.argtypes = [i64, i64, i64]
+    lib.oracle_scale_bits_per_weight.restype = dbl
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _setup(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+def use_library(path):
+    """Point this module at another build of dbf_oracle.c (used by the tests that
+    plant mistakes in a copy of the oracle); returns the previous library."""
+    global _lib
+    prev = _lib
+    _lib = _setup(ctypes.CDLL(path)) if path is not None else None
+    return prev
+
+
+def restore_library(prev):
+    global _lib
+    _lib = prev
+
+
+def _f64(a) -> np.ndarray:
+    # fp16 -> fp64 widening is exact.
+    return np.ascontiguousarray(np.asarray(a), dtype=np.float64)
+
+
+def _i8(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a), dtype=np.int8)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def words_per_row(cols: int) -> int:
+    """32-bit words per packed row (rows are padded to 128 bits)."""
+    return int(_load().oracle_words_per_row(cols))
+
+
+def unpack_signs(packed, rows: int, cols: int):
+    """Decode the documented packed layout into int8 +-1 (rows x cols).
+
+    Returns (signs, n_set_padding_bits)."""
+    lib = _load()
+    packed = np.ascontiguousarray(np.asarray(packed), dtype=np.uint32).reshape(-1)
+    if packed.size < rows * words_per_row(cols):
+        raise ValueError("packed buffer too small")
+    out = np.empty((rows, cols), dtype=np.int8)
+    bad = lib.oracle_unpack_signs(_ptr(packed), rows, cols, _ptr(out))
+    return out, int(bad)
+
+
+def pack_signs(signs) -> np.ndarray:
+    """Encode int8 signs (< 0 -> set bit) into the documented packed layout."""
+    lib = _load()
+    s = _i8(signs)
+    rows, cols = s.shape
+    out = np.empty(rows * words_per_row(cols), dtype=np.uint32)
+    lib.oracle_pack_signs(_ptr(s), rows, cols, _ptr(out))
+    return out
+
+
+def forward_staged(x, A, B, a, mid, b, return_v: bool = False):
+    """((((x (.) b) B^T) (.) mid) A^T) (.) a in fp64 (section 2.1, computation process).
+
+    x: batch x m_in; A: n x k signs; B: k x m_in signs; a: n; mid: k; b: m_in.
+    Returns y (batch x n), and v = mid (.) (B (x (.) b)) (batch x k) if asked."""
+    lib = _load()
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    A, B = _i8(A), _i8(B)
+    a, mid, b = _f64(a), _f64(mid), _f64(b)
+    n, k = A.shape
+    k2, m_in = B.shape
+    batch = x.shape[0]
+    if k2 != k or x.shape[1] != m_in or a.size != n or mid.size != k or b.size != m_in:
+        raise ValueError("shape mismatch")
+    y = np.empty((batch, n), dtype=np.float64)
+    v = np.empty((batch, k), dtype=np.float64) if return_v else None
+    lib.oracle_forward_staged(_ptr(x), _ptr(A), _ptr(B), _ptr(a), _ptr(mid), _ptr(b), n, k, m_in,
+                              batch, _ptr(y), _ptr(v) if v is not None else None)
+    return (y, v) if return_v else y
+
+
+def dense_weight(A, B, a, mid, b) -> np.ndarray:
+    """W = (a (.) A (.) mid^T)(B (.) b^T), n x m_in, fp64 (section 2.1, factorisation)."""
+    lib = _load()
+    A, B = _i8(A), _i8(B)
+    a, mid, b = _f64(a), _f64(mid), _f64(b)
+    n, k = A.shape
+    m_in = B.shape[1]
+    if B.shape[0] != k or a.size != n or mid.size != k or b.size != m_in:
+        raise ValueError("shape mismatch")
+    W = np.empty((n, m_in), dtype=np.float64)
+    lib.oracle_dense_weight(_ptr(A), _ptr(B), _ptr(a), _ptr(mid), _ptr(b), n, k, m_in, _ptr(W))
+    return W
+
+
+def forward_dense(x, W) -> np.ndarray:
+    """y = x W^T with a dense fp64 W."""
+    lib = _load()
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    W = _f64(W)
+    n, m_in = W.shape
+    y = np.empty((x.shape[0], n), dtype=np.float64)
+    lib.oracle_forward_dense(_ptr(x), _ptr(W), n, m_in, x.shape[0], _ptr(y))
+    return y
+
+
+def bits_per_weight(n: int, k: int, m_in: int) -> float:
+    """Sign bits per dense weight, k(n + m_in)/(n m_in) (section 2.1: k sets the rate)."""
+    return float(_load().oracle_bits_per_weight(n, k, m_in))
+
+
+def scale_bits_per_weight(n: int, k: int, m_in: int) -> float:
+    """fp16 scale-vector bits per dense weight, 16(n + k + m_in)/(n m_in)."""
+    return float(_load().oracle_scale_bits_per_weight(n, k, m_in))

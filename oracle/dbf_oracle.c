@@ -1,0 +1,188 @@
+/*
+ * fp64 CPU oracle for the Double Binary Factorization (DBF) layer.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only tests/, __graft_entry__.smoke()
+ * and bench.py's cpu_baseline / reference leg may load this library.  It shares
+ * no source, header, table or helper with the CUDA path in
+ * binary_factorized_weight_b200/ and neither side includes or calls the other.
+ *
+ * Source: "Addition is almost all you need: Compressing large language models
+ * with double binary factorization" (gist.science technical summary, section
+ * 2.1 "mathematical formulation"; sciencestack.ai abstract and Figure 1).
+ *
+ *   factorisation  W ~= (a (.) A (.) m^T)(B (.) b^T),  A in {+-1}^(n x k),
+ *                  B in {+-1}^(k x m_in), a, m, b fp16 vectors   (section 2.1)
+ *   evaluation     X W^T ~= ((((X (.) b^T) B^T) (.) m^T) A^T) (.) a^T
+ *                  every product with a sign matrix is additions and sign
+ *                  flips                                      (section 2.1,
+ *                                                  "computation process")
+ *
+ * Everything is computed in fp64 from inputs that the caller has widened
+ * exactly from fp16 / +-1.  The method has no approximation at inference time,
+ * so the oracle is the plain definition written out with loops; no blocking,
+ * fusion or reordering beyond the evaluation order above.
+ *
+ * Packed sign layout decoded by oracle_unpack_signs (the pages only say the
+ * matrices are binary/sign; the bit layout is this library's own choice):
+ *   - a rows x cols sign matrix is stored row after row; each row takes
+ *     ceil(cols/128)*4 little-endian 32-bit words (a multiple of 16 bytes);
+ *   - element c of a row lives in word c/32; inside that word, element
+ *     e = c%32 sits at bit (e/2) + 16*(e%2): even elements fill bits 0..15,
+ *     odd elements bits 16..31;
+ *   - a set bit means -1, a clear bit +1; bits past the last column are 0.
+ *
+ * Parity status of each function (see the test-suite pins in
+ * tests/test_oracle_pins.py):
+ *   oracle_forward_staged, oracle_dense_weight, oracle_forward_dense,
+ *   oracle_unpack_signs, oracle_pack_signs, oracle_bits_per_weight: pinned.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* Words per packed row: the row is padded to a multiple of 128 bits. */
+int64_t oracle_words_per_row(int64_t cols) { return ((cols + 127) / 128) * 4; }
+
+/* Bit position of element e (0..31) inside its 32-bit word. */
+static int bit_of_element(int e) { return (e >> 1) + ((e & 1) << 4); }
+
+/*
+ * Decode a packed sign matrix into int8 +-1 values (row-major rows x cols).
+ * Returns the number of set padding bits found (0 for a valid buffer).
+ */
+int64_t oracle_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out) {
+  const int64_t wpr = oracle_words_per_row(cols);
+  int64_t bad_padding = 0;
+  for (int64_t r = 0; r < rows; ++r) {
+    const uint32_t* row = packed + r * wpr;
+    for (int64_t c = 0; c < cols; ++c) {
+      uint32_t word = row[c / 32];
+      int bit = bit_of_element((int)(c % 32));
+      out[r * cols + c] = ((word >> bit) & 1u) ? (int8_t)-1 : (int8_t)1;
+    }
+    for (int64_t c = cols; c < wpr * 32; ++c) {
+      uint32_t word = row[c / 32];
+      int bit = bit_of_element((int)(c % 32));
+      bad_padding += (word >> bit) & 1u;
+    }
+  }
+  return bad_padding;
+}
+
+/*
+ * Encode int8 signs into the packed layout.  An entry < 0 becomes a set bit;
+ * 0 and positive entries become clear bits.
+ */
+void oracle_pack_signs(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* packed) {
+  const int64_t wpr = oracle_words_per_row(cols);
+  memset(packed, 0, (size_t)(rows * wpr) * sizeof(uint32_t));
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) {
+      if (signs[r * cols + c] < 0) {
+        packed[r * wpr + c / 32] |= 1u << bit_of_element((int)(c % 32));
+      }
+    }
+  }
+}
+
+/*
+ * Staged forward, in the order of the "computation process" equation:
+ *   u = x (.) b                (X (.) b^T)
+ *   t = B u                    (. B^T, additions and sign flips)
+ *   v = mid (.) t              ((.) m^T)
+ *   z = A v                    (. A^T, additions and sign flips)
+ *   y = a (.) z                ((.) a^T)
+ * x is batch x m_in, y is batch x n, A is n x k, B is k x m_in (row-major int8).
+ * If v_out is non-NULL it receives v (batch x k).
+ */
+void oracle_forward_staged(const double* x, const int8_t* A, const int8_t* B, const double* a,
+                           const double* mid, const double* b, int64_t n, int64_t k, int64_t m_in,
+                           int64_t batch, double* y, double* v_out) {
+  double* ubuf = (double*)malloc((size_t)m_in * sizeof(double));
+  double* vbuf = (double*)malloc((size_t)k * sizeof(double));
+  if (!ubuf || !vbuf) {
+    free(ubuf);
+    free(vbuf);
+    for (int64_t e = 0; e < batch * n; ++e) y[e] = NAN;
+    return;
+  }
+  for (int64_t tok = 0; tok < batch; ++tok) {
+    const double* xt = x + tok * m_in;
+    for (int64_t j = 0; j < m_in; ++j) ubuf[j] = xt[j] * b[j];
+#pragma omp parallel for schedule(static)
+    for (int64_t l = 0; l < k; ++l) {
+      const int8_t* Bl = B + l * m_in;
+      double acc = 0.0;
+      for (int64_t j = 0; j < m_in; ++j) acc += (double)Bl[j] * ubuf[j];
+      vbuf[l] = mid[l] * acc;
+    }
+    if (v_out) memcpy(v_out + tok * k, vbuf, (size_t)k * sizeof(double));
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+      const int8_t* Ai = A + i * k;
+      double acc = 0.0;
+      for (int64_t l = 0; l < k; ++l) acc += (double)Ai[l] * vbuf[l];
+      y[tok * n + i] = a[i] * acc;
+    }
+  }
+  free(ubuf);
+  free(vbuf);
+}
+
+/*
+ * Dense reconstruction W = (a (.) A (.) m^T)(B (.) b^T), n x m_in:
+ *   W[i][j] = sum_l (a_i A[i][l] m_l) (B[l][j] b_j)
+ */
+void oracle_dense_weight(const int8_t* A, const int8_t* B, const double* a, const double* mid,
+                         const double* b, int64_t n, int64_t k, int64_t m_in, double* W) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    double* Wi = W + i * m_in;
+    for (int64_t j = 0; j < m_in; ++j) Wi[j] = 0.0;
+    for (int64_t l = 0; l < k; ++l) {
+      const double left = a[i] * (double)A[i * k + l] * mid[l];
+      const int8_t* Bl = B + l * m_in;
+      for (int64_t j = 0; j < m_in; ++j) Wi[j] += left * ((double)Bl[j] * b[j]);
+    }
+  }
+}
+
+/* y = x W^T for a dense W (n x m_in); x is batch x m_in. */
+void oracle_forward_dense(const double* x, const double* W, int64_t n, int64_t m_in, int64_t batch,
+                          double* y) {
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t tok = 0; tok < batch; ++tok) {
+    for (int64_t i = 0; i < n; ++i) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < m_in; ++j) acc += x[tok * m_in + j] * W[i * m_in + j];
+      y[tok * n + i] = acc;
+    }
+  }
+}
+
+/*
+ * Storage cost.  Section 2.1 names the middle dimension k as the knob that
+ * sets the compression rate (section 2.3 builds the per-layer allocation on
+ * it).  Sign bits per dense weight: k(n + m_in)/(n m_in).
+ * The three fp16 scale vectors add 16(n + k + m_in)/(n m_in).
+ */
+double oracle_bits_per_weight(int64_t n, int64_t k, int64_t m_in) {
+  return (double)k * (double)(n + m_in) / ((double)n * (double)m_in);
+}
+
+double oracle_scale_bits_per_weight(int64_t n, int64_t k, int64_t m_in) {
+  return 16.0 * (double)(n + k + m_in) / ((double)n * (double)m_in);
+}

@@ -1,0 +1,85 @@
+"""Plant plausible mistakes in copies of the oracle and check the pins catch each.
+
+Each mutant is the oracle's C source with one edit (a dropped scale, a wrong
+sign, a transposed or reversed operand, a dropped term, a wrong bit layout),
+compiled into a temporary library on the CPU.  The pins of
+test_oracle_pins.py are then run against the mutant; at least one must fail.
+This shows the pins are strong enough to trust the unmutated oracle.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "dbf_oracle.c")
+
+MUTANTS = {
+    "drop_b": ("ubuf[j] = xt[j] * b[j];", "ubuf[j] = xt[j];"),
+    "drop_mid": ("vbuf[l] = mid[l] * acc;", "vbuf[l] = acc;"),
+    "drop_a": ("y[tok * n + i] = a[i] * acc;", "y[tok * n + i] = acc;"),
+    "wrong_sign_B": ("acc += (double)Bl[j] * ubuf[j];", "acc -= (double)Bl[j] * ubuf[j];"),
+    "transposed_A": ("acc += (double)Ai[l] * vbuf[l];", "acc += (double)A[l * n + i] * vbuf[l];"),
+    "reversed_B": ("acc += (double)Bl[j] * ubuf[j];", "acc += (double)Bl[m_in - 1 - j] * ubuf[j];"),
+    "dropped_last_term": ("for (int64_t l = 0; l < k; ++l) acc += (double)Ai[l]",
+                          "for (int64_t l = 0; l + 1 < k; ++l) acc += (double)Ai[l]"),
+    "mid_indexed_by_row": ("vbuf[l] = mid[l] * acc;", "vbuf[l] = mid[l % (k > 1 ? k - 1 : 1)] * acc;"),
+    "natural_bit_layout": ("return (e >> 1) + ((e & 1) << 4);", "return e;"),
+    "dense_drops_b": ("Wi[j] += left * ((double)Bl[j] * b[j]);", "Wi[j] += left * ((double)Bl[j]);"),
+    "dense_transposed_B": ("Wi[j] += left * ((double)Bl[j] * b[j]);",
+                           "Wi[j] += left * ((double)B[(j % k) * m_in + (l % m_in)] * b[j]);"),
+    "bpw_off": ("return (double)k * (double)(n + m_in) / ((double)n * (double)m_in);",
+                "return (double)k * (double)(n + m_in) / ((double)n * (double)(m_in + 1));"),
+}
+
+PIN_CHECKS = [
+    lambda o: pins.test_hand_worked_example(o),
+    lambda o: pins.test_exhaustive_2x2x2(o),
+    lambda o: pins.test_brute_force_fractions(o, 3, 2, 5),
+    lambda o: pins.test_staged_equals_dense(o, 96, 64, 320, 2),
+    lambda o: pins.test_integer_mode_is_exact(o),
+    lambda o: pins.test_hadamard_closed_form(o, 3),
+    lambda o: pins.test_k1_outer_product(o),
+    lambda o: pins.test_orientation_is_not_transposed(o),
+    lambda o: pins.test_bits_per_weight_closed_form(o, 4096, 2048, 4096, 1.0),
+    lambda o: pins.test_layout_table(o),
+    lambda o: pins.test_layout_round_trip_and_padding(o, 3, 128),
+]
+
+
+def _build_mutant(name, tmpdir):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found; update the mutant table"
+    path_c = os.path.join(tmpdir, f"{name}.c")
+    path_so = os.path.join(tmpdir, f"{name}.so")
+    with open(path_c, "w") as f:
+        f.write(src.replace(old, new, 1))
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", path_so, path_c, "-lm"],
+                   check=True)
+    return path_so
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    with tempfile.TemporaryDirectory() as tmpdir:
+        so = _build_mutant(name, tmpdir)
+        prev = oracle.use_library(so)
+        caught = []
+        try:
+            for i, check in enumerate(PIN_CHECKS):
+                try:
+                    check(oracle)
+                except AssertionError:
+                    caught.append(i)
+        finally:
+            oracle.restore_library(prev)
+    assert caught, f"no pin caught mutant {name}"
+
+
+def test_unmutated_oracle_passes_all_checks():
+    for check in PIN_CHECKS:
+        check(oracle)

@@ -1,0 +1,297 @@
+"""Pins for the fp64 oracle: each check ties it to something other than itself.
+
+Sources of truth used here (none of them calls the oracle's C code):
+  * a forward worked by hand (tests/golden/worked_example_2x2x3.txt);
+  * exact integer arithmetic (numpy int64 / Python Fractions) on tiny shapes,
+    exhaustively at n = k = m_in = 2;
+  * the Sylvester-Hadamard closed form: with A = B = H_k, H_k H_k = k I, and the
+    staged product equals a (.) FWHT(mid (.) FWHT(b (.) x)), with a butterfly
+    FWHT written here;
+  * the k = 1 rank-one closed form;
+  * invariances of the factorisation (sign moves, middle permutation);
+  * the bits/weight closed form against packed byte counts;
+  * the documented packed layout table (tests/golden/packed_layout_bits.txt).
+The factorisation and evaluation order follow "Addition is almost all you
+need", gist.science technical summary section 2.1.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import dbf_inputs as gen
+from conftest import read_golden
+
+
+# ---------------------------------------------------------------- worked example
+def test_hand_worked_example(oracle_mod):
+    g = read_golden("worked_example_2x2x3.txt")
+    n, k, m_in = int(g["n"][0]), int(g["k"][0]), int(g["m_in"][0])
+    A = np.array(g["A"], dtype=np.int8).reshape(n, k)
+    B = np.array(g["B"], dtype=np.int8).reshape(k, m_in)
+    x = np.array(g["x"]).reshape(1, m_in)
+    y = oracle_mod.forward_staged(x, A, B, g["a"], g["mid"], g["b"])
+    assert y.tolist() == [g["y"]]
+    W = oracle_mod.dense_weight(A, B, g["a"], g["mid"], g["b"])
+    assert W.reshape(-1).tolist() == g["W"]
+    assert oracle_mod.forward_dense(x, W).tolist() == [g["y"]]
+
+
+# ---------------------------------------------------------------- exact integer brute force
+def _exact_int_forward(x, A, B, a, mid, b):
+    """y = x W^T with W = diag(a) A diag(mid) B diag(b), all in int64."""
+    W = (a[:, None] * A.astype(np.int64) * mid[None, :]) @ (B.astype(np.int64) * b[None, :])
+    return x.astype(np.int64) @ W.T
+
+
+def test_exhaustive_2x2x2(oracle_mod):
+    """Every 2x2 sign pair (2^8 patterns) times every x in {-2..2}^2, integer scales."""
+    xs = np.array([[p, q] for p in range(-2, 3) for q in range(-2, 3)], dtype=np.int64)
+    a = np.array([3, -2], dtype=np.int64)
+    mid = np.array([2, 5], dtype=np.int64)
+    b = np.array([-1, 4], dtype=np.int64)
+    for pattern in range(256):
+        bits = [(pattern >> i) & 1 for i in range(8)]
+        A = np.array([1 - 2 * v for v in bits[:4]], dtype=np.int8).reshape(2, 2)
+        B = np.array([1 - 2 * v for v in bits[4:]], dtype=np.int8).reshape(2, 2)
+        y = oracle_mod.forward_staged(xs, A, B, a, mid, b)
+        assert np.array_equal(y, _exact_int_forward(xs, A, B, a, mid, b).astype(np.float64)), pattern
+
+
+@pytest.mark.parametrize("n,k,m_in", [(1, 1, 1), (3, 2, 5), (5, 7, 3), (8, 4, 8), (2, 8, 6)])
+def test_brute_force_fractions(oracle_mod, n, k, m_in):
+    """Non-integer fp16-exact scales: compare to exact rational arithmetic."""
+    rng = np.random.default_rng(17 + n * 100 + k * 10 + m_in)
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    a = gen.abs_normal_scales(rng, n)
+    mid = -gen.abs_normal_scales(rng, k)  # negative scales are legal too
+    b = gen.abs_normal_scales(rng, m_in)
+    x = gen.normal_activations(rng, 3, m_in)
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    F = lambda v: Fraction(float(v))  # fp16 -> float is exact, float -> Fraction is exact
+    for t in range(3):
+        for i in range(n):
+            exact = sum(
+                F(a[i]) * int(A[i, l]) * F(mid[l]) * int(B[l, j]) * F(b[j]) * F(x[t, j])
+                for l in range(k)
+                for j in range(m_in)
+            )
+            got = y[t, i]
+            assert abs(Fraction(got) - exact) <= abs(exact) * Fraction(1, 10**12) + Fraction(1, 10**30)
+
+
+# ---------------------------------------------------------------- associativity
+@pytest.mark.parametrize("n,k,m_in,batch", [(256, 128, 256, 3), (96, 64, 320, 2), (40, 192, 64, 5)])
+def test_staged_equals_dense(oracle_mod, n, k, m_in, batch):
+    """Staged evaluation (computation process) vs dense reconstruction (factorisation)."""
+    rng = np.random.default_rng(n + k + m_in)
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    a, mid, b = gen.lognormal_scales(rng, n), gen.abs_normal_scales(rng, k), gen.lognormal_scales(rng, m_in)
+    x = gen.normal_activations(rng, batch, m_in)
+    y_staged = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    y_dense = oracle_mod.forward_dense(x, oracle_mod.dense_weight(A, B, a, mid, b))
+    rel = np.linalg.norm(y_staged - y_dense) / np.linalg.norm(y_dense)
+    assert rel < 1e-12
+    # and against numpy's own matmul of the dense factors
+    xf = x.astype(np.float64)
+    W_np = (a.astype(np.float64)[:, None] * A * mid.astype(np.float64)[None, :]) @ (B * b.astype(np.float64)[None, :])
+    rel_np = np.linalg.norm(y_staged - xf @ W_np.T) / np.linalg.norm(y_staged)
+    assert rel_np < 1e-12
+
+
+# ---------------------------------------------------------------- integer invariant
+def test_integer_mode_is_exact(oracle_mod):
+    shape = gen.CONFIGS["tiny_int"]
+    L = gen.make_layer(shape, batch=4)
+    y = oracle_mod.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])
+    assert np.all(y == np.round(y))
+    one_n, one_k, one_m = (np.ones(s, dtype=np.int64) for s in (shape.n, shape.k, shape.m_in))
+    exact = _exact_int_forward(L["x"].astype(np.int64), L["A"], L["B"], one_n, one_k, one_m)
+    assert np.array_equal(y, exact.astype(np.float64))
+    # the middle vector stays inside fp16's exact-integer range for this recipe
+    _, v = oracle_mod.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"], return_v=True)
+    assert np.abs(v).max() <= 2048
+
+
+# ---------------------------------------------------------------- Hadamard closed form
+def _fwht(v):
+    """Unnormalised Walsh-Hadamard transform in Sylvester order, butterfly form, last axis."""
+    v = np.array(v, dtype=np.float64, copy=True)
+    h = 1
+    size = v.shape[-1]
+    while h < size:
+        v = v.reshape(v.shape[:-1] + (size // (2 * h), 2, h))
+        lo, hi = v[..., 0, :].copy(), v[..., 1, :].copy()
+        v[..., 0, :], v[..., 1, :] = lo + hi, lo - hi
+        v = v.reshape(v.shape[:-3] + (size,))
+        h *= 2
+    return v
+
+
+def test_sylvester_pattern_matches_scipy():
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    for p in range(0, 7):
+        assert np.array_equal(gen.sylvester_hadamard(p), scipy_linalg.hadamard(1 << p).astype(np.int8))
+
+
+@pytest.mark.parametrize("p", [1, 3, 6, 8])
+def test_hadamard_closed_form(oracle_mod, p):
+    size = 1 << p
+    H = gen.sylvester_hadamard(p)
+    rng = np.random.default_rng(p)
+    x = gen.integer_activations(rng, 3, size)
+    ones = np.ones(size, dtype=np.float16)
+    # unit scales: H H = size * I, so y = size * x exactly
+    y = oracle_mod.forward_staged(x, H, H, ones, ones, ones)
+    assert np.array_equal(y, size * x.astype(np.float64))
+    # general scales: y = a (.) FWHT(mid (.) FWHT(b (.) x))
+    a, mid, b = gen.abs_normal_scales(rng, size), gen.lognormal_scales(rng, size), gen.abs_normal_scales(rng, size)
+    xn = gen.normal_activations(rng, 3, size)
+    y = oracle_mod.forward_staged(xn, H, H, a, mid, b)
+    closed = a.astype(np.float64) * _fwht(mid.astype(np.float64) * _fwht(b.astype(np.float64) * xn.astype(np.float64)))
+    assert np.allclose(y, closed, rtol=1e-12, atol=1e-12 * np.abs(closed).max())
+
+
+# ---------------------------------------------------------------- rank-one closed form
+def test_k1_outer_product(oracle_mod):
+    rng = np.random.default_rng(5)
+    n, m_in = 37, 53
+    A = gen.sign_matrix(rng, n, 1)
+    B = gen.sign_matrix(rng, 1, m_in)
+    a, mid, b = gen.lognormal_scales(rng, n), gen.abs_normal_scales(rng, 1), gen.abs_normal_scales(rng, m_in)
+    x = gen.integer_activations(rng, 4, m_in)
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    inner = x.astype(np.float64) @ (B[0].astype(np.float64) * b.astype(np.float64))  # <B[0,:], b (.) x>
+    closed = np.outer(inner * float(mid[0]), a.astype(np.float64) * A[:, 0])
+    assert np.allclose(y, closed, rtol=1e-14, atol=0)
+
+
+# ---------------------------------------------------------------- invariances
+def _layer(seed, n=48, k=64, m_in=80, batch=3):
+    rng = np.random.default_rng(seed)
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    x = gen.integer_activations(rng, batch, m_in)
+    a = rng.integers(-3, 4, n).astype(np.float16)
+    mid = rng.integers(-3, 4, k).astype(np.float16)
+    b = rng.integers(-3, 4, m_in).astype(np.float16)
+    return x, A, B, a, mid, b
+
+
+def test_invariance_row_sign_move(oracle_mod):
+    x, A, B, a, mid, b = _layer(1)
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    A2, a2 = A.copy(), a.copy()
+    A2[[3, 7, 11]] *= -1
+    a2[[3, 7, 11]] *= -1
+    assert np.array_equal(oracle_mod.forward_staged(x, A2, B, a2, mid, b), y)
+
+
+def test_invariance_middle_sign_move(oracle_mod):
+    x, A, B, a, mid, b = _layer(2)
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    cols = [0, 5, 63]
+    A2, B2 = A.copy(), B.copy()
+    A2[:, cols] *= -1
+    B2[cols, :] *= -1
+    assert np.array_equal(oracle_mod.forward_staged(x, A2, B2, a, mid, b), y)
+    mid2 = mid.copy()
+    mid2[cols] *= -1
+    A3 = A.copy()
+    A3[:, cols] *= -1
+    assert np.array_equal(oracle_mod.forward_staged(x, A3, B, a, mid2, b), y)
+
+
+def test_invariance_middle_permutation(oracle_mod):
+    x, A, B, a, mid, b = _layer(3)
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    perm = np.random.default_rng(9).permutation(A.shape[1])
+    assert np.array_equal(oracle_mod.forward_staged(x, A[:, perm], B[perm, :], a, mid[perm], b), y)
+
+
+def test_orientation_is_not_transposed(oracle_mod):
+    """b scales inputs (columns of B), a scales outputs (rows of A): check with one-hot scales."""
+    x, A, B, a, mid, b = _layer(4, n=6, k=4, m_in=9, batch=1)
+    x = np.ones((1, 9), dtype=np.float16)
+    a = np.ones(6, dtype=np.float16)
+    mid = np.ones(4, dtype=np.float16)
+    b = np.zeros(9, dtype=np.float16)
+    b[2] = 1  # only input column 2 survives
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    assert np.array_equal(y[0], (A.astype(np.float64) @ B[:, 2].astype(np.float64)))
+    a = np.zeros(6, dtype=np.float16)
+    a[4] = 1  # only output row 4 survives
+    b = np.ones(9, dtype=np.float16)
+    y = oracle_mod.forward_staged(x, A, B, a, mid, b)
+    expect = np.zeros(6)
+    expect[4] = A[4].astype(np.float64) @ B.astype(np.float64).sum(axis=1)
+    assert np.array_equal(y[0], expect)
+
+
+# ---------------------------------------------------------------- bits per weight
+@pytest.mark.parametrize(
+    "n,k,m_in,expect",
+    [(4096, 2048, 4096, 1.0), (4096, 4096, 4096, 2.0), (14336, 4736, 4096, 4736 * 18432 / (14336 * 4096)),
+     (256, 128, 256, 1.0)],
+)
+def test_bits_per_weight_closed_form(oracle_mod, n, k, m_in, expect):
+    assert oracle_mod.bits_per_weight(n, k, m_in) == pytest.approx(expect, rel=1e-15)
+    # packed sign storage: rows are 128-aligned here, so bits = k*n + k*m_in exactly
+    words = n * oracle_mod.words_per_row(k) + k * oracle_mod.words_per_row(m_in)
+    assert words * 32 / (n * m_in) == pytest.approx(expect, rel=1e-15)
+    assert oracle_mod.scale_bits_per_weight(n, k, m_in) == pytest.approx(16 * (n + k + m_in) / (n * m_in))
+
+
+def test_bits_per_weight_rounding_rule():
+    """k for a target bit rate: nearest multiple of 64, ties up (layer set recipe)."""
+    def k_for(n, m_in, bits):
+        exact = bits * n * m_in / (n + m_in)
+        return int(np.floor(exact / 64 + 0.5)) * 64
+
+    for bits, shapes in gen.LAYER_SET.items():
+        for s in shapes:
+            assert s.k == k_for(s.n, s.m_in, bits), s.name
+
+
+# ---------------------------------------------------------------- packed layout
+def test_layout_table(oracle_mod):
+    table = read_golden("packed_layout_bits.txt")
+    for e_str, (bit,) in table.items():
+        e = int(e_str)
+        signs = np.ones((1, 32), dtype=np.int8)
+        signs[0, e] = -1
+        packed = oracle_mod.pack_signs(signs)
+        assert packed.tolist() == [1 << int(bit), 0, 0, 0]
+        back, bad = oracle_mod.unpack_signs(np.array([1 << int(bit), 0, 0, 0], dtype=np.uint32), 1, 32)
+        assert bad == 0 and np.array_equal(back, signs)
+
+
+def test_layout_hand_words(oracle_mod):
+    # 0x0000FFFF: bits 0..15 set -> even elements are -1, odd are +1
+    back, bad = oracle_mod.unpack_signs(np.array([0x0000FFFF, 0, 0, 0], dtype=np.uint32), 1, 32)
+    assert bad == 0
+    assert back[0].tolist() == [-1 if e % 2 == 0 else 1 for e in range(32)]
+    # second word of a row holds elements 32..63; rows are 4 words apart for cols <= 128
+    packed = np.zeros(8, dtype=np.uint32)
+    packed[1] = 1 << 16  # element 33
+    packed[4 + 3] = 1 << 31  # row 1, element 127
+    back, bad = oracle_mod.unpack_signs(packed, 2, 128)
+    assert bad == 0
+    assert [int(i) for i in np.nonzero(back[0] < 0)[0]] == [33]
+    assert [int(i) for i in np.nonzero(back[1] < 0)[0]] == [127]
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 64), (3, 128), (5, 192), (17, 320), (2, 1000)])
+def test_layout_round_trip_and_padding(oracle_mod, rows, cols):
+    rng = np.random.default_rng(rows * cols)
+    s = gen.sign_matrix(rng, rows, cols)
+    packed = oracle_mod.pack_signs(s)
+    assert packed.size == rows * ((cols + 127) // 128) * 4
+    back, bad = oracle_mod.unpack_signs(packed, rows, cols)
+    assert bad == 0 and np.array_equal(back, s)
+    if cols % 128:
+        corrupt = packed.copy()
+        corrupt[((cols + 127) // 128) * 4 - 1] |= np.uint32(1 << 31)  # last padding bit of row 0
+        assert oracle_mod.unpack_signs(corrupt, rows, cols)[1] == 1
