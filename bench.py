@@ -1,0 +1,515 @@
+"""Benchmark of the DBF layer forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload attn_1b] [--batch 1] [--sweep OUT.json]
+
+Workload (default): the Llama-8B-shaped attention projection n = m_in = 4096,
+k = 2048 (1.0 bit/weight), batch 1 (config attn_1b of dbf_inputs).  A step is
+the forward of one batch through R distinct copies of that layer (each copy in
+its own HBM buffers, R * bytes >= 4 * L2), so every layer's weights stream from
+HBM; the R forwards are captured once as a CUDA graph and the graph is replayed
+once per step.  Metric: tokens/s through one DBF layer (= batch / time per
+layer forward), with us/layer and achieved HBM GB/s reported alongside.
+
+Multi-GPU (torchrun, N > 1): replicas only - every rank runs the same workload
+on its own GPU with no data-path collective; the timed region is bracketed by
+barriers and the slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import dbf_inputs as gen  # noqa: E402
+
+METRIC = "DBF layer fwd µs, HBM GB/s (% of peak) & tokens/s at 1/2 bit, batch 1–2048"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def layer_bytes(n, k, m_in, batch):
+    """Algorithmic HBM bytes of one layer forward: packed signs, fp16 scales, x in, y out."""
+    return n * k / 8 + k * m_in / 8 + 2 * (n + k + m_in) + 2 * batch * (m_in + n)
+
+
+def layer_flops(n, k, m_in, batch):
+    """Signed additions of the two sign products, counted as multiply-adds (2 flops)."""
+    return 2.0 * batch * k * (m_in + n)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "binary_factorized_weight_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload_key):
+    """DRAM bytes per forward from the committed ncu summary, if the kernels are unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        entry = t[workload_key]
+        if entry.get("source_hash") != kernel_source_hash():
+            return None
+        return entry["dram_bytes_per_forward"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if not inside:
+            inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
+            window = "nearest samples (timed region shorter than the sampling period)"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ reference arm (the fp64 oracle)
+def oracle_rate(shape, batch, seconds, rotation=0):
+    """Time the oracle as it stands on host cores: tokens/s through one layer."""
+    import oracle
+
+    L = gen.make_layer(shape, batch, rotation)
+    oracle.forward_staged(L["x"][:1], L["A"], L["B"], L["a"], L["mid"], L["b"])  # load + page in
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return batch * calls / el, calls, el, oracle.num_threads()
+
+
+def run_reference(args, shape, batch):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    import oracle
+
+    L = gen.make_layer(shape, batch)
+    oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])  # warm
+    for _ in range(args.warmup):
+        oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])
+    el = time.perf_counter() - t0
+    value = batch * args.steps / el
+    sample = f"one layer forward ({shape.name}, batch {batch}) per step out of the R-layer step of the GPU arm"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(shape, batch), "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def workload_name(shape, batch):
+    bpw = shape.k * (shape.n + shape.m_in) / (shape.n * shape.m_in)
+    return f"{shape.name}: n={shape.n} m_in={shape.m_in} k={shape.k} ({bpw:.3f} bit/weight), batch {batch}"
+
+
+# ------------------------------------------------------------------ our arm
+class Workload:
+    """R rotated copies of one layer on the device plus everything a step needs."""
+
+    def __init__(self, dbf, torch, shape, batch, device, copies=None, flags=None):
+        self.dbf, self.torch = dbf, torch
+        self.shape, self.batch = shape, batch
+        n, k, m_in = shape.n, shape.k, shape.m_in
+        L = gen.make_layer(shape, batch)
+        self.host = L
+        d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        pA = dbf.dbf_pack_signs(d(L["A"]))
+        pB = dbf.dbf_pack_signs(d(L["B"]))
+        a, mid, b = d(L["a"]), d(L["mid"]), d(L["b"])
+        self.bytes = layer_bytes(n, k, m_in, batch)
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        weight_bytes = (pA.numel() + pB.numel()) * 4 + 2 * (n + k + m_in)
+        self.copies = copies or max(2, int(math.ceil(4 * l2 / weight_bytes)))
+        self.pA = [pA] + [pA.clone() for _ in range(self.copies - 1)]
+        self.pB = [pB] + [pB.clone() for _ in range(self.copies - 1)]
+        self.sc = [(a, mid, b)] + [(a.clone(), mid.clone(), b.clone()) for _ in range(self.copies - 1)]
+        self.x = d(L["x"])
+        self.y = torch.empty((batch, n), dtype=torch.float16, device=device)
+        self.ws = dbf.dbf_new_workspace(n, k, m_in, batch, device=device)
+        self.flags = dbf.DBF_FWD_WEIGHTS_STATIC if flags is None else flags
+        self.weight_bytes_total = self.copies * weight_bytes
+        decode = batch <= 16 and not (self.flags & dbf.DBF_FWD_FORCE_PREFILL)
+        self.launches_per_forward = 2 * (math.ceil(batch / 16) if decode else 1)
+        self.path = "decode (mma.sync sign-GEMV, 2 PDL-chained stages)" if decode else "prefill (tcgen05, 2 GEMMs)"
+
+    def forward_all(self, x=None, y=None):
+        x = self.x if x is None else x
+        y = self.y if y is None else y
+        s = self.shape
+        for i in range(self.copies):
+            a, mid, b = self.sc[i]
+            self.dbf.dbf_forward(x, self.pA[i], self.pB[i], a, mid, b, s.n, s.k, s.m_in, y=y, workspace=self.ws,
+                                 flags=self.flags)
+
+    def capture(self):
+        torch = self.torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward_all()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward_all()
+        torch.cuda.synchronize()
+        return g
+
+
+def run_ours(args, shape, batch):
+    import torch
+
+    world, rank, local = dist_setup(args)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+
+    from binary_factorized_weight_b200 import build as lib_build
+
+    lib_build.build()
+    import binary_factorized_weight_b200 as dbf
+
+    dbf.load_library()
+    peaks = load_peaks()
+    wl = Workload(dbf, torch, shape, batch, device)
+    graph = wl.capture()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---------------------------------------------------------- device-timed steps
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    ev0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    ms_per_step = ms / args.steps
+    us_per_layer = 1e3 * ms_per_step / wl.copies
+    tokens_per_s = world * batch / (us_per_layer * 1e-6)
+    hbm_gbs = wl.bytes / (us_per_layer * 1e-6) / 1e9
+
+    # ---------------------------------------------------------- end to end: host buffers, copies inside
+    x_host = torch.from_numpy(np.ascontiguousarray(wl.host["x"])).pin_memory()
+    y_host = torch.empty((batch, shape.n), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty_like(wl.x)
+    g2 = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        wl.forward_all(x=x_dev)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g2):
+        wl.forward_all(x=x_dev)
+    torch.cuda.synchronize()
+    e2e_steps = max(1, args.steps)
+    for _ in range(max(3, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        g2.replay()
+        y_host.copy_(wl.y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        g2.replay()
+        y_host.copy_(wl.y, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * batch * wl.copies * e2e_steps / (e2e_ms * 1e-3)
+
+    # output check of the timed configuration (sampled, against the oracle)
+    check = None
+    if rank == 0 and args.check:
+        import oracle
+
+        torch.cuda.synchronize()
+        ref = oracle.forward_staged(wl.host["x"], wl.host["A"], wl.host["B"], wl.host["a"], wl.host["mid"],
+                                    wl.host["b"])
+        y = y_host.float().numpy().astype(np.float64)
+        check = float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+
+    if world > 1:
+        torch.distributed.barrier()
+        del graph, g2
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    # ---------------------------------------------------------- CPU baseline (oracle), rank 0 at N = 1 only
+    cpu = None
+    if world == 1 and args.cpu_seconds > 0:
+        rate, calls, el, cores = oracle_rate(shape, batch, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{calls} fp64 oracle forwards of one {shape.name} layer at batch {batch} "
+                         f"({el:.1f} s on host cores)"}
+
+    key = f"{shape.name}_b{batch}"
+    traffic = traffic_for(key)
+    result = {
+        "metric": METRIC,
+        "value": tokens_per_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": workload_name(shape, batch),
+            "path": wl.path,
+            "layers_per_step": wl.copies,
+            "l2": f"inputs larger than L2: {wl.copies} distinct weight copies, "
+                  f"{wl.weight_bytes_total / 1e6:.0f} MB >= 4 x L2",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "graph": "one CUDA graph of the step's dbf_forward calls, replayed once per step",
+        },
+        "us_per_layer": us_per_layer,
+        "hbm_gbs": hbm_gbs,
+        "hbm_frac": hbm_gbs / peaks["hbm_gbs"],
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "dbf_forward decode pair (stage B + stage A, PDL-overlapped, one layer)",
+            "achieved": hbm_gbs,
+            "peak": peaks["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": hbm_gbs / peaks["hbm_gbs"],
+            "traffic": traffic,
+            "peak_source": f"{peaks['source']} (STREAM-style copy, MEASURED_PEAKS.json)",
+            "algorithmic_bytes_per_layer": wl.bytes,
+        },
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2)},
+        "gpu_launches": args.steps * wl.copies * wl.launches_per_forward,
+        "clocks": clocks,
+    }
+    if batch > 16:
+        fl = layer_flops(shape.n, shape.k, shape.m_in, batch)
+        tf = fl / (us_per_layer * 1e-6) / 1e12
+        result["roofline"] = {
+            "bound": "tensor", "kernel": "dbf_forward prefill pair (GEMM1 + GEMM2, one layer)", "achieved": tf,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "traffic": traffic,
+            "peak_source": f"{peaks['source']} dense bf16 burst (fp16 runs at the bf16 rate)",
+            "algorithmic_flops_per_layer": fl}
+    if check is not None:
+        result["output_check_rel_fro"] = check
+    print(json.dumps(result))
+
+
+# ------------------------------------------------------------------ sweep (all configs, one GPU)
+def run_sweep(args):
+    import torch
+
+    torch.cuda.set_device(0)
+    from binary_factorized_weight_b200 import build as lib_build
+
+    lib_build.build()
+    import binary_factorized_weight_b200 as dbf
+
+    dbf.load_library()
+    peaks = load_peaks()
+    device = torch.device("cuda", 0)
+    cases = [(gen.CONFIGS["attn_1b"], 1)]
+    cases += [(gen.CONFIGS["attn_2b"], b) for b in (1, 4, 16)]
+    cases += [(gen.CONFIGS["mlp_up"], b) for b in (1, 2048)]
+    for bits in (1, 2):
+        for s in gen.LAYER_SET[bits]:
+            cases += [(s, b) for b in (1, 16, 128, 2048)]
+    rows = []
+    for shape, batch in cases:
+        wl = Workload(dbf, torch, shape, batch, device)
+        g = wl.capture()
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = max(3, int(200 / max(1, wl.copies)))
+        times = []
+        for _ in range(7):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / reps / wl.copies * 1e3)
+        us = statistics.median(times)
+        gbs = wl.bytes / (us * 1e-6) / 1e9
+        tf = layer_flops(shape.n, shape.k, shape.m_in, batch) / (us * 1e-6) / 1e12
+        row = {"layer": shape.name, "n": shape.n, "k": shape.k, "m_in": shape.m_in, "batch": batch,
+               "bpw": shape.k * (shape.n + shape.m_in) / (shape.n * shape.m_in), "us": us,
+               "us_p10": sorted(times)[0], "us_p90": sorted(times)[-1], "tokens_per_s": batch / (us * 1e-6),
+               "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": tf,
+               "tensor_frac": tf / peaks["bf16_tflops"], "copies": wl.copies, "path": wl.path}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del g, wl
+        torch.cuda.empty_cache()
+    with open(args.sweep, "w") as f:
+        json.dump({"peaks": peaks, "rows": rows}, f, indent=1)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="attn_1b", choices=sorted(gen.CONFIGS))
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-check", dest="check", action="store_false")
+    ap.add_argument("--sweep", default=None, help="run every config and write a JSON table here")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    shape = gen.CONFIGS[args.workload]
+    if args.sweep:
+        run_sweep(args)
+    elif args.impl == "reference":
+        run_reference(args, shape, args.batch)
+    else:
+        run_ours(args, shape, args.batch)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+"""DBF (Double Binary Factorization) layer forward on B200: Python binding.
+
+A thin ctypes binding of ``libdbf.so`` (C ABI in ``include/dbf.h``).  Every
+function here only marshals torch tensors into pointers, sizes and the current
+CUDA stream; all computation runs in the library's sm_100a kernels.  There is
+no CPU or library fallback: if ``libdbf.so`` is missing the import of the
+binding's functions raises, and a call on a machine without a B200 returns the
+library's error as :class:`DBFError`.
+
+    y = W x with W = (a (.) A (.) m^T)(B (.) b^T)  ("Addition is almost all you
+    need", gist.science technical summary section 2.1), evaluated as
+    ((((x (.) b) B^T) (.) m) A^T) (.) a without forming W.
+
+Build the library with ``python -m binary_factorized_weight_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "DBFError",
+    "DBF_I8", "DBF_F16", "DBF_F32",
+    "DBF_FWD_WEIGHTS_STATIC", "DBF_FWD_FORCE_DECODE", "DBF_FWD_FORCE_PREFILL", "DBF_FWD_DECODE_SHIFT_EXPAND",
+    "EXPORTED_SYMBOLS",
+    "library_path", "load_library",
+    "dbf_packed_words_per_row", "dbf_packed_words", "dbf_pack_signs",
+    "dbf_forward_workspace_bytes", "dbf_new_workspace", "dbf_forward",
+    "dbf_reconstruct_dense", "dbf_workspace_status", "dbf_status_string",
+]
+
+DBF_I8, DBF_F16, DBF_F32 = 0, 1, 2
+DBF_FWD_WEIGHTS_STATIC = 1 << 0
+DBF_FWD_FORCE_DECODE = 1 << 1
+DBF_FWD_FORCE_PREFILL = 1 << 2
+DBF_FWD_DECODE_SHIFT_EXPAND = 1 << 3
+
+STATUS_NAMES = {
+    0: "DBF_OK", 1: "DBF_ERR_INVALID_ARG", 2: "DBF_ERR_UNSUPPORTED_SHAPE", 3: "DBF_ERR_MISALIGNED",
+    4: "DBF_ERR_WORKSPACE", 5: "DBF_ERR_CUDA", 6: "DBF_ERR_TIMEOUT", 7: "DBF_ERR_DEVICE",
+}
+
+EXPORTED_SYMBOLS = (
+    "dbf_packed_words_per_row",
+    "dbf_packed_words",
+    "dbf_pack_signs",
+    "dbf_forward_workspace_bytes",
+    "dbf_forward",
+    "dbf_reconstruct_dense",
+    "dbf_workspace_status",
+    "dbf_status_string",
+)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+class DBFError(RuntimeError):
+    def __init__(self, func: str, status: int):
+        self.status = status
+        super().__init__(f"{func} failed: {dbf_status_string(status)}")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libdbf.so")
+
+
+def load_library():
+    """Load libdbf.so (built in-tree) and declare its signatures."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m binary_factorized_weight_b200.build`")
+    lib = ctypes.CDLL(path)
+    i64, u32, i32, vp, sz = ctypes.c_int64, ctypes.c_uint32, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    lib.dbf_packed_words_per_row.argtypes = [i64]
+    lib.dbf_packed_words_per_row.restype = i64
+    lib.dbf_packed_words.argtypes = [i64, i64]
+    lib.dbf_packed_words.restype = i64
+    lib.dbf_pack_signs.argtypes = [vp, i32, i64, i64, vp, vp]
+    lib.dbf_pack_signs.restype = i32
+    lib.dbf_forward_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.dbf_forward_workspace_bytes.restype = sz
+    lib.dbf_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, vp, sz, u32, vp]
+    lib.dbf_forward.restype = i32
+    lib.dbf_reconstruct_dense.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, i32, vp]
+    lib.dbf_reconstruct_dense.restype = i32
+    lib.dbf_workspace_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.dbf_workspace_status.restype = i32
+    lib.dbf_status_string.argtypes = [i32]
+    lib.dbf_status_string.restype = ctypes.c_char_p
+    _LIB = lib
+    return lib
+
+
+def _check(func: str, status: int):
+    if status != 0:
+        raise DBFError(func, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(dtype: torch.dtype) -> int:
+    if dtype == torch.int8:
+        return DBF_I8
+    if dtype == torch.float16:
+        return DBF_F16
+    if dtype == torch.float32:
+        return DBF_F32
+    raise TypeError(f"unsupported dtype {dtype}")
+
+
+def dbf_status_string(status: int) -> str:
+    try:
+        return load_library().dbf_status_string(int(status)).decode()
+    except ImportError:
+        return STATUS_NAMES.get(int(status), "unknown dbf_status")
+
+
+def dbf_packed_words_per_row(cols: int) -> int:
+    return int(load_library().dbf_packed_words_per_row(int(cols)))
+
+
+def dbf_packed_words(rows: int, cols: int) -> int:
+    return int(load_library().dbf_packed_words(int(rows), int(cols)))
+
+
+def dbf_pack_signs(src: torch.Tensor, packed: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pack a rows x cols sign matrix (int8/fp16/fp32 CUDA tensor; < 0 -> -1).
+
+    Returns an int32 CUDA tensor holding the packed 32-bit words."""
+    if src.dim() != 2 or not src.is_contiguous():
+        raise ValueError("src must be a contiguous 2-D tensor")
+    rows, cols = src.shape
+    n_words = dbf_packed_words(rows, cols)
+    if packed is None:
+        packed = torch.empty(n_words, dtype=torch.int32, device=src.device)
+    elif packed.numel() < n_words or packed.dtype != torch.int32:
+        raise ValueError("packed must be an int32 tensor of dbf_packed_words(rows, cols) words")
+    _check("dbf_pack_signs", load_library().dbf_pack_signs(
+        _ptr(src), _dtype_code(src.dtype), rows, cols, _ptr(packed), _stream(stream)))
+    return packed
+
+
+def dbf_forward_workspace_bytes(n: int, k: int, m_in: int, batch: int) -> int:
+    return int(load_library().dbf_forward_workspace_bytes(int(n), int(k), int(m_in), int(batch)))
+
+
+def dbf_new_workspace(n: int, k: int, m_in: int, batch: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size dbf_forward needs (uint8 CUDA tensor)."""
+    return torch.zeros(dbf_forward_workspace_bytes(n, k, m_in, batch), dtype=torch.uint8, device=device)
+
+
+def dbf_forward(x: torch.Tensor, packedA: torch.Tensor, packedB: torch.Tensor, a: torch.Tensor, m: torch.Tensor,
+                b: torch.Tensor, n: int, k: int, m_in: int, y: Optional[torch.Tensor] = None,
+                y_dtype: torch.dtype = torch.float16, workspace: Optional[torch.Tensor] = None, flags: int = 0,
+                stream=None) -> torch.Tensor:
+    """y = ((((x (.) b) B^T) (.) m) A^T) (.) a for fp16 x (batch x m_in); returns y (batch x n)."""
+    if x.dtype != torch.float16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp16 batch x m_in tensor")
+    batch = x.shape[0]
+    if x.shape[1] != m_in:
+        raise ValueError("x.shape[1] != m_in")
+    if y is None:
+        y = torch.empty((batch, n), dtype=y_dtype, device=x.device)
+    if workspace is None:
+        workspace = dbf_new_workspace(n, k, m_in, batch, device=x.device)
+    y_code = _dtype_code(y.dtype)
+    _check("dbf_forward", load_library().dbf_forward(
+        _ptr(x), _ptr(packedA), _ptr(packedB), _ptr(a), _ptr(m), _ptr(b), int(n), int(k), int(m_in), int(batch),
+        _ptr(y), y_code, _ptr(workspace), workspace.numel() * workspace.element_size(), int(flags), _stream(stream)))
+    return y
+
+
+def dbf_reconstruct_dense(packedA: torch.Tensor, packedB: torch.Tensor, a: torch.Tensor, m: torch.Tensor,
+                          b: torch.Tensor, n: int, k: int, m_in: int, W: Optional[torch.Tensor] = None,
+                          W_dtype: torch.dtype = torch.float32, stream=None) -> torch.Tensor:
+    """Dense W = (a (.) A (.) m^T)(B (.) b^T), n x m_in."""
+    if W is None:
+        W = torch.empty((n, m_in), dtype=W_dtype, device=a.device)
+    _check("dbf_reconstruct_dense", load_library().dbf_reconstruct_dense(
+        _ptr(packedA), _ptr(packedB), _ptr(a), _ptr(m), _ptr(b), int(n), int(k), int(m_in), _ptr(W),
+        _dtype_code(W.dtype), _stream(stream)))
+    return W
+
+
+def dbf_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """The workspace's device status word (0, or the dbf_status of the first device-side failure)."""
+    out = ctypes.c_int32(0)
+    _check("dbf_workspace_status", load_library().dbf_workspace_status(
+        _ptr(workspace), _stream(stream), ctypes.byref(out)))
+    return int(out.value)

@@ -1,0 +1,293 @@
+// Prefill path (large batches): one sign-product GEMM per launch on the
+// fifth-generation tensor cores (tcgen05, accumulator in tensor memory).
+//
+// Same product as the decode stage ("Addition is almost all you need",
+// gist.science technical summary, section 2.1, computation process):
+//
+//   out[tok][row] = rowscale[row] * sum_K sign(row, K) * kscale[K] * act[tok][K]
+//
+// GEMM1: rows = k, K = m_in, kscale = b, act = x, rowscale = mid, out = V (fp16)
+// GEMM2: rows = n, K = k,    no kscale,  act = V, rowscale = a,   out = y
+//
+// The tile computes D[128 weight rows x NTILE tokens] = S * act^T, i.e. the
+// weights are the M operand.  That makes each expanded sign tile serve NTILE
+// tokens (expansion work per flop halves against tokens-as-M), puts one weight
+// row in each TMEM lane so the epilogue scale (mid or a) is a per-thread
+// scalar, and lets the epilogue write 32 consecutive rows of an output token
+// per warp store.
+//
+// Roles (192 threads):
+//   warps 0-3  sign expansion: thread r turns row r's 64 packed bits of a K step
+//              into 64 fp16 values (+-1, or +-b_j with b folded in by flipping
+//              the scale's sign bit: exact) and stores them as one 128-byte row
+//              of a 128B-swizzled K-major tile; later the epilogue (TMEM ->
+//              registers -> scaled global stores).
+//   warp 4     TMA producer of the activation tile (K-major, 128B swizzle,
+//              out-of-range tokens read as zero).
+//   warp 5     TMEM allocation and the single-thread tcgen05.mma issue loop.
+// Stage hand-off is through mbarriers; every wait is bounded and an expired
+// wait records DBF_ERR_TIMEOUT in the workspace status word, raises a CTA-wide
+// abort flag and lets all roles fall through to the teardown, which frees TMEM
+// only after this thread's MMAs are known to be complete.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "dbf_device.cuh"
+#include "dbf_internal.h"
+
+namespace dbf {
+namespace {
+
+constexpr int kBM = 128;  // weight rows per tile (TMEM lanes)
+constexpr int kBK = 64;   // K per pipeline stage: one 128-byte swizzle row of fp16
+constexpr int kThreads = 192;
+constexpr int kABytes = kBM * kBK * 2;
+
+template <int NTILE>
+struct Cfg {
+  static constexpr int kStages = NTILE == 256 ? 4 : 6;
+  static constexpr int kBBytes = NTILE * kBK * 2;
+  static constexpr int kBarOffset = kStages * (kABytes + kBBytes);
+  // full_a[S], full_b[S], empty[S], acc_full, mma_done
+  static constexpr int kNumBars = 3 * kStages + 2;
+  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;  // + tmem slot/abort + align slack
+};
+
+template <int NTILE, bool KSCALE, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+    dbf_prefill_gemm_kernel(const __grid_constant__ CUtensorMap act_map, const PrefillArgs p) {
+  using C = Cfg<NTILE>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_st = smem;
+  uint8_t* b_st = smem + S * kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* full_a = bars;
+  uint64_t* full_b = bars + S;
+  uint64_t* empty = bars + 2 * S;
+  uint64_t* acc_full = bars + 3 * S;
+  uint64_t* mma_done = bars + 3 * S + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int m_tiles = (p.M + kBM - 1) / kBM;
+  const int m0 = (blockIdx.x % m_tiles) * kBM;
+  const int n0 = (blockIdx.x / m_tiles) * NTILE;
+  const int KT = p.K / kBK;
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_a[i], 128);
+      mbar_init(&full_b[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) prefetch_tmap(&act_map);
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, NTILE);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp < 4) {
+    // ------------------------------------------------ sign expansion
+    const int r = m0 + tid;
+    const bool rok = r < p.M;
+    const uint2* wrow = reinterpret_cast<const uint2*>(p.packed + (rok ? static_cast<int64_t>(r) * p.wpr : 0));
+    uint2 wnext = make_uint2(0u, 0u);
+    if (p.weights_early && rok) wnext = __ldg(wrow);
+    pdl_wait();
+    if (!p.weights_early && rok) wnext = __ldg(wrow);
+    bool ok = true;
+    const int swz = tid & 7;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % S;
+      const uint32_t use = static_cast<uint32_t>(kt / S);
+      const uint2 wcur = wnext;
+      if (kt + 1 < KT && rok) wnext = __ldg(wrow + kt + 1);
+      if (kt >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      uint8_t* dst = a_st + s * kABytes + (tid >> 3) * 1024 + swz * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t wsel = (j < 4) ? wcur.x : wcur.y;
+        uint32_t h[4];
+        if constexpr (KSCALE) {
+          const uint4 sc = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 8 * j));
+          h[0] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 0, sc.x);
+          h[1] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 1, sc.y);
+          h[2] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 2, sc.z);
+          h[3] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 3, sc.w);
+        } else {
+          h[0] = pm1_pair_rt(wsel, 4 * (j & 3) + 0);
+          h[1] = pm1_pair_rt(wsel, 4 * (j & 3) + 1);
+          h[2] = pm1_pair_rt(wsel, 4 * (j & 3) + 2);
+          h[3] = pm1_pair_rt(wsel, 4 * (j & 3) + 3);
+        }
+        *reinterpret_cast<uint4*>(dst + ((j ^ swz) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&full_a[s]);
+    }
+
+    // ------------------------------------------------ epilogue
+    if (ok && mbar_wait_bounded(acc_full, 0, abort_flag, p.status)) {
+      tc_fence_after();
+      const int row = m0 + warp * 32 + lane;
+      const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;
+      for (int col = 0; col < NTILE; col += 32) {
+        if (n0 + col >= p.batch) break;  // warp-uniform
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(col), v);
+        tmem_ld_wait();
+        if (row < p.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = n0 + col + j;
+            if (tok < p.batch) {
+              const float val = rs * __uint_as_float(v[j]);
+              if constexpr (OUT_F32) {
+                static_cast<float*>(p.out)[static_cast<int64_t>(tok) * p.ld_out + row] = val;
+              } else {
+                static_cast<__half*>(p.out)[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(val);
+              }
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      pdl_wait();
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % S;
+        const uint32_t use = static_cast<uint32_t>(kt / S);
+        if (kt >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&full_b[s], C::kBBytes);
+        tma_load_2d(b_st + s * C::kBBytes, &act_map, kt * kBK, n0, &full_b[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------ MMA issue
+    if (lane == 0) {
+      pdl_wait();
+      constexpr uint32_t idesc = idesc_f16_f32(kBM, NTILE);
+      bool ok = true;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        const int s = kt % S;
+        const uint32_t par = static_cast<uint32_t>(kt / S) & 1;
+        if (!mbar_wait_bounded(&full_a[s], par, abort_flag, p.status) ||
+            !mbar_wait_bounded(&full_b[s], par, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(a_st + s * kABytes);
+        const uint32_t b_addr = smem_u32(b_st + s * C::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          tc_mma_f16_ss(tmem_d, smem_desc_sw128_kmajor(a_addr + kk * 32), smem_desc_sw128_kmajor(b_addr + kk * 32),
+                        idesc, (kt | kk) != 0 ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      if (ok) tc_commit(acc_full);
+      tc_commit(mma_done);
+    }
+  }
+
+  // ------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    // Free TMEM once every MMA this CTA issued has finished (the wait is
+    // bounded; TMEM must be released before the CTA exits either way).
+    (void)mbar_wait_bounded(mma_done, 0, abort_flag, p.status);
+    __syncwarp();
+    tmem_dealloc(tmem_d, NTILE);
+  }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+  });
+  return fn;
+}
+
+template <int NTILE, bool KSCALE, bool OUT_F32>
+dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, const DeviceInfo& dev, cudaStream_t stream) {
+  (void)dev;
+  auto kernel = dbf_prefill_gemm_kernel<NTILE, KSCALE, OUT_F32>;
+  constexpr int smem = Cfg<NTILE>::kSmemBytes;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DBF_ERR_CUDA;
+  const int64_t m_tiles = (a.M + kBM - 1) / kBM;
+  const int64_t n_tiles = (a.batch + NTILE - 1) / NTILE;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(m_tiles * n_tiles), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, map, a) == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
+}
+
+}  // namespace
+
+dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t act_rows, bool out_f32,
+                               const DeviceInfo& dev, cudaStream_t stream) {
+  auto encode = encode_fn();
+  if (!encode) return DBF_ERR_CUDA;
+  const int ntile = a.batch > 128 ? 256 : 128;
+  if (static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + ntile - 1) / ntile) > 0x7fffffffLL)
+    return DBF_ERR_UNSUPPORTED_SHAPE;
+
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(act_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(ntile)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(act), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return DBF_ERR_CUDA;
+
+  const bool ks = a.kscale != nullptr;
+  if (ntile == 256) {
+    if (ks) return out_f32 ? launch_typed<256, true, true>(a, map, dev, stream) : launch_typed<256, true, false>(a, map, dev, stream);
+    return out_f32 ? launch_typed<256, false, true>(a, map, dev, stream) : launch_typed<256, false, false>(a, map, dev, stream);
+  }
+  if (ks) return out_f32 ? launch_typed<128, true, true>(a, map, dev, stream) : launch_typed<128, true, false>(a, map, dev, stream);
+  return out_f32 ? launch_typed<128, false, true>(a, map, dev, stream) : launch_typed<128, false, false>(a, map, dev, stream);
+}
+
+}  // namespace dbf

@@ -1,0 +1,186 @@
+/*
+ * dbf.h — C ABI of libdbf, a single-GPU (B200, sm_100a) implementation of the
+ * Double Binary Factorization (DBF) linear-layer forward pass.
+ *
+ * The method ("Addition is almost all you need: Compressing large language
+ * models with double binary factorization"; gist.science technical summary,
+ * section 2.1; sciencestack.ai Figure 1) replaces a dense weight W (n x m_in) by
+ *
+ *     W ~= (a (.) A (.) mid^T)(B (.) b^T)
+ *
+ * with A in {+-1}^(n x k), B in {+-1}^(k x m_in) and fp16 scale vectors a (n),
+ * mid (k), b (m_in).  ("mid" is the middle vector the pages call m; it is named
+ * m in the argument lists below.)  The forward of an input batch X is evaluated
+ * in the order the pages give, so that both sign products are additions and
+ * sign flips:
+ *
+ *     Y = X W^T ~= ((((X (.) b^T) B^T) (.) mid^T) A^T) (.) a^T
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All data pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or keeps memory and keeps no state between calls.
+ *  - fp16 buffers are IEEE binary16 bit patterns (uint16_t), e.g. __half or a
+ *    torch.float16 tensor.
+ *  - Matrices are row-major and dense (no padding between rows) unless said.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  A call returns after enqueueing.
+ *  - Synchronous argument checks run first; a call that returns anything but
+ *    DBF_OK has enqueued nothing.  DBF_ERR_CUDA reports a failed launch; faults
+ *    that happen later on the device surface through the stream (and, for
+ *    dbf_forward, the workspace status word, see dbf_workspace_status).
+ *  - No C++ exception crosses this interface.
+ *
+ * Packed sign layout (the pages only say the factors are binary sign
+ * matrices; this bit layout is the library's own choice):
+ *  - A rows x cols sign matrix is stored row after row.  Each row occupies
+ *    dbf_packed_words_per_row(cols) = ceil(cols/128)*4 little-endian 32-bit
+ *    words, so every row starts on a 16-byte boundary.
+ *  - Element c of a row is held in word c/32 of that row, at bit
+ *    (e/2) + 16*(e%2) with e = c%32: the even elements of the 32-element group
+ *    fill bits 0..15 and the odd elements bits 16..31.  Element pair (2q, 2q+1)
+ *    therefore sits at bits (q, q+16), the two sign positions of an fp16 pair
+ *    after one shift.
+ *  - A set bit means -1, a clear bit +1.  Bits past the last column are 0.
+ *  - packedA holds A (n rows over k columns); packedB holds B (k rows over
+ *    m_in columns): both are packed along the reduction dimension of their
+ *    product.
+ */
+#ifndef DBF_H_
+#define DBF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* the type a cudaStream_t points to */
+
+#if defined(__GNUC__)
+#define DBF_API __attribute__((visibility("default")))
+#else
+#define DBF_API
+#endif
+
+typedef enum dbf_status {
+  DBF_OK = 0,
+  DBF_ERR_INVALID_ARG = 1,       /* null pointer, negative size, unknown enum, bad flag */
+  DBF_ERR_UNSUPPORTED_SHAPE = 2, /* outside the shape contract of the call */
+  DBF_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  DBF_ERR_WORKSPACE = 4,         /* workspace null, misaligned or smaller than required */
+  DBF_ERR_CUDA = 5,              /* a CUDA runtime call or kernel launch failed */
+  DBF_ERR_TIMEOUT = 6,           /* a bounded device-side wait gave up (status word) */
+  DBF_ERR_DEVICE = 7             /* the current device is not an sm_100 (B200-class) GPU */
+} dbf_status;
+
+typedef enum dbf_dtype { DBF_I8 = 0, DBF_F16 = 1, DBF_F32 = 2 } dbf_dtype;
+
+/* dbf_forward flags (bitwise OR; 0 is the safe default). */
+enum {
+  /* The packed signs and the three scale vectors are not written by any work
+   * that may still be running on `stream` when this call is enqueued (true for
+   * inference weights loaded ahead of time).  The kernels may then start
+   * streaming weights before the previous kernel on the stream has finished
+   * (programmatic dependent launch).  x is always read only after it. */
+  DBF_FWD_WEIGHTS_STATIC = 1u << 0,
+  /* Force the batch <= 16 sign-GEMV path (batches above 16 run in chunks of 16). */
+  DBF_FWD_FORCE_DECODE = 1u << 1,
+  /* Force the tensor-core (tcgen05) path at any batch size. */
+  DBF_FWD_FORCE_PREFILL = 1u << 2,
+  /* Decode path: form the fp16 sign operands by shift+mask with one
+   * accumulator set instead of the default bit-position classes. */
+  DBF_FWD_DECODE_SHIFT_EXPAND = 1u << 3
+};
+
+/* Words (uint32) in one packed row of `cols` signs: ceil(cols/128)*4.
+ * Returns 0 for cols <= 0. */
+DBF_API int64_t dbf_packed_words_per_row(int64_t cols);
+
+/* Words (uint32) of a packed rows x cols sign matrix: rows*ceil(cols/128)*4.
+ * Returns 0 for rows <= 0 or cols <= 0. */
+DBF_API int64_t dbf_packed_words(int64_t rows, int64_t cols);
+
+/*
+ * Pack a sign matrix into the layout above (the pages' storage format: A and
+ * B hold only +-1 entries, sciencestack.ai Figure 1; gist.science section 2.1).
+ *   src     rows x cols, row-major, element type src_t (DBF_I8, DBF_F16 or
+ *           DBF_F32).  An element packs to -1 (set bit) iff it compares < 0;
+ *           0, -0.0 and NaN pack to +1.
+ *   packed  dbf_packed_words(rows, cols) words, written in full (padding bits
+ *           are cleared).  Must be 16-byte aligned and must not overlap src.
+ * Shape: rows >= 1, cols >= 1.  Any cols is accepted here; dbf_forward itself
+ * needs k and m_in to be multiples of 64.
+ */
+DBF_API dbf_status dbf_pack_signs(const void* src, dbf_dtype src_t, int64_t rows, int64_t cols,
+                          uint32_t* packed, struct CUstream_st* stream);
+
+/*
+ * Workspace bytes dbf_forward needs for these sizes (0 if a size is < 1).
+ * Layout: a 256-byte status block (an int32 status word at offset 0), then
+ * the middle activations V = fp16(mid (.) (B (x (.) b))) as batch x k fp16.
+ * The workspace must be zero-filled before its first use; the library leaves
+ * the status word untouched unless a device-side wait gives up.  Calls that
+ * may run concurrently need distinct workspaces.
+ */
+DBF_API size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, int64_t batch);
+
+/*
+ * y = ((((x (.) b^T) B^T) (.) m^T) A^T) (.) a^T    (section 2.1, computation
+ * process; both sign products are evaluated without materialising W).
+ *
+ *   x          batch x m_in fp16, row-major.
+ *   packedA    A in the packed layout, n rows over k.
+ *   packedB    B in the packed layout, k rows over m_in.
+ *   a, m, b    fp16 vectors of n, k and m_in entries (m is the pages' middle
+ *              vector, "mid" above).
+ *   y          batch x n, row-major, y_t = DBF_F16 (round to nearest even,
+ *              overflow to +-inf) or DBF_F32.
+ *   workspace  ws_bytes >= dbf_forward_workspace_bytes(n, k, m_in, batch),
+ *              zero-filled before its first use (see above).
+ *   flags      DBF_FWD_* bits.
+ * Arithmetic: both sign products accumulate in fp32.  The middle vector V is
+ * rounded to fp16 once (V = fp16(mid (.) t)); the decode path also rounds
+ * x (.) b to fp16 before the first product, the tensor-core path folds b into
+ * the sign operand exactly.  With a = m = b = 1, integer x and |t| <= 2048,
+ * every step is exact and fp32 output equals the integer result.
+ * Paths: batch <= 16 runs two PDL-chained sign-GEMV kernels (mma.sync);
+ * larger batches run two tcgen05 tensor-core kernels.
+ * Shape contract: n >= 1, batch >= 1, k and m_in multiples of 64 in
+ * [64, 1 << 20], n and batch <= 1 << 24.  All pointers 16-byte aligned;
+ * outputs must not overlap inputs.
+ */
+DBF_API dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB,
+                       const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n, int64_t k,
+                       int64_t m_in, int64_t batch, void* y, dbf_dtype y_t, void* workspace,
+                       size_t ws_bytes, uint32_t flags, struct CUstream_st* stream);
+
+/*
+ * Dense reconstruction W = (a (.) A (.) m^T)(B (.) b^T), n x m_in row-major
+ * (section 2.1, factorisation equation):
+ *     W[i][j] = a_i * b_j * sum_l A[i][l] m_l B[l][j]   (fp32 accumulation)
+ * W_t is DBF_F16 (round to nearest even) or DBF_F32.  Not a hot path: it
+ * exists to check a factorisation against the dense weight it stands for.
+ * Shape contract as dbf_forward (k, m_in multiples of 64); pointers 16-byte
+ * aligned.
+ */
+DBF_API dbf_status dbf_reconstruct_dense(const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
+                                 const uint16_t* m, const uint16_t* b, int64_t n, int64_t k, int64_t m_in,
+                                 void* W, dbf_dtype W_t, struct CUstream_st* stream);
+
+/*
+ * Copy the workspace status word to *device_status (synchronises `stream`).
+ * 0 means no device-side wait has given up since the workspace was zeroed;
+ * otherwise it holds the dbf_status of the first failure (DBF_ERR_TIMEOUT).
+ */
+DBF_API dbf_status dbf_workspace_status(const void* workspace, struct CUstream_st* stream, int32_t* device_status);
+
+/* Static, NUL-terminated description of a status code. */
+DBF_API const char* dbf_status_string(dbf_status status);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* DBF_H_ */

@@ -1,0 +1,127 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol that
+include/dbf.h declares, and rejects bad arguments before touching a device.
+
+No test here launches a kernel or needs a GPU.  Pointers passed to calls that
+must fail validation are never dereferenced (validation returns first).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import binary_factorized_weight_b200 as dbf
+from binary_factorized_weight_b200 import build as dbf_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dbf.h")
+
+OK, INVALID, SHAPE, MISALIGNED, WORKSPACE, CUDA_ERR = 0, 1, 2, 3, 4, 5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dbf_build.build()
+    return dbf.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*DBF_API\s+(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(dbf_[a-z_]+)\s*\(", text,
+                       flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_api():
+    names = declared_functions()
+    assert set(names) == set(dbf.EXPORTED_SYMBOLS), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_packed_words(lib):
+    assert dbf.dbf_packed_words_per_row(1) == 4
+    assert dbf.dbf_packed_words_per_row(128) == 4
+    assert dbf.dbf_packed_words_per_row(129) == 8
+    assert dbf.dbf_packed_words_per_row(4096) == 128
+    assert dbf.dbf_packed_words(4096, 2048) == 4096 * 64
+    assert dbf.dbf_packed_words(0, 64) == 0
+    assert dbf.dbf_packed_words(3, -1) == 0
+
+
+def test_workspace_bytes(lib):
+    assert dbf.dbf_forward_workspace_bytes(4096, 2048, 4096, 1) == 256 + 4096
+    assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 4) == 256 + 1024
+    assert dbf.dbf_forward_workspace_bytes(256, 64, 256, 1) == 256 + 256  # V padded to 256 bytes
+    assert dbf.dbf_forward_workspace_bytes(0, 128, 256, 4) == 0
+
+
+def test_status_strings(lib):
+    for code, name in dbf.STATUS_NAMES.items():
+        assert dbf.dbf_status_string(code).startswith(name)
+    assert "unknown" in dbf.dbf_status_string(99)
+
+
+# fake, never-dereferenced device addresses
+P = 1 << 20  # 16-byte aligned
+MIS = P + 2
+
+
+def fwd(lib, x=P, A=P, B=P, a=P, m=P, b=P, n=256, k=128, m_in=256, batch=4, y=P, y_t=1, ws=P, ws_bytes=1 << 20,
+        flags=0):
+    return lib.dbf_forward(x, A, B, a, m, b, n, k, m_in, batch, y, y_t, ws, ws_bytes, flags, None)
+
+
+@pytest.mark.parametrize(
+    "kwargs,expect",
+    [
+        (dict(x=None), INVALID), (dict(A=None), INVALID), (dict(B=None), INVALID), (dict(a=None), INVALID),
+        (dict(m=None), INVALID), (dict(b=None), INVALID), (dict(y=None), INVALID),
+        (dict(n=0), INVALID), (dict(batch=0), INVALID), (dict(batch=-3), INVALID), (dict(k=0), INVALID),
+        (dict(k=96), SHAPE), (dict(m_in=100), SHAPE), (dict(k=1 << 21), SHAPE), (dict(n=(1 << 24) + 1), SHAPE),
+        (dict(batch=(1 << 24) + 1), SHAPE),
+        (dict(y_t=0), INVALID), (dict(y_t=7), INVALID),
+        (dict(flags=1 << 9), INVALID), (dict(flags=2 | 4), INVALID),
+        (dict(x=MIS), MISALIGNED), (dict(A=MIS), MISALIGNED), (dict(B=MIS), MISALIGNED),
+        (dict(a=MIS), MISALIGNED), (dict(y=MIS), MISALIGNED),
+        (dict(ws=None), WORKSPACE), (dict(ws=MIS), WORKSPACE), (dict(ws_bytes=256 + 1023), WORKSPACE),
+    ],
+)
+def test_forward_validation(lib, kwargs, expect):
+    assert fwd(lib, **kwargs) == expect
+
+
+def test_forward_valid_args_without_device(lib):
+    """Valid arguments on a machine with no usable B200 must fail cleanly, not crash."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; covered by the gpu tests")
+    assert fwd(lib) in (CUDA_ERR, 7)
+
+
+def test_pack_validation(lib):
+    assert lib.dbf_pack_signs(None, 0, 4, 64, P, None) == INVALID
+    assert lib.dbf_pack_signs(P, 0, 4, 64, None, None) == INVALID
+    assert lib.dbf_pack_signs(P, 5, 4, 64, P, None) == INVALID
+    assert lib.dbf_pack_signs(P, 0, 0, 64, P, None) == INVALID
+    assert lib.dbf_pack_signs(P, 0, 4, 64, MIS, None) == MISALIGNED
+    assert lib.dbf_pack_signs(P + 1, 2, 4, 64, P, None) == MISALIGNED  # fp32 source not 4-byte aligned
+
+
+def test_reconstruct_validation(lib):
+    assert lib.dbf_reconstruct_dense(P, P, P, P, P, 256, 128, 256, None, 2, None) == INVALID
+    assert lib.dbf_reconstruct_dense(P, P, P, P, P, 256, 100, 256, P, 2, None) == SHAPE
+    assert lib.dbf_reconstruct_dense(P, P, P, P, P, 256, 128, 256, P, 0, None) == INVALID
+    assert lib.dbf_reconstruct_dense(P, P, P, P, P, 256, 128, 256, MIS, 2, None) == MISALIGNED
+
+
+def test_workspace_status_validation(lib):
+    out = ctypes.c_int32()
+    assert lib.dbf_workspace_status(None, None, ctypes.byref(out)) == INVALID
+    assert lib.dbf_workspace_status(P, None, None) == INVALID
