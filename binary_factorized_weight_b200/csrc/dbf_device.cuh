@@ -38,26 +38,33 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// Bit position of element e (0..31) inside its packed 32-bit word: element
-// pair (2q, 2q+1) lives at bits (q, q+16).
-__device__ __forceinline__ int packed_bit_of(int e) { return (e >> 1) + ((e & 1) << 4); }
+// Packed layout: rows of ceil(cols/256) blocks of 8 words.  Column e of a
+// block (0..255) is in group e/16 and pair (e%16)/2; it lives in word
+// (e%16)/2 of the block at bit (e/16) + 16*(e%2).  Word p of a block therefore
+// holds, at bits (g, g+16), the column pair (16g + 2p, 16g + 2p + 1).
+__device__ __forceinline__ int packed_word_in_block(int e) { return (e & 15) >> 1; }
+__device__ __forceinline__ int packed_bit_in_block(int e) { return (e >> 4) + ((e & 1) << 4); }
 
-// fp16 pair (+-1, +-1) for element pair q of word w: shift bits (q, q+16) to the
-// two fp16 sign positions (15, 31) and OR them into the pair (1.0, 1.0).
-template <int Q>
-__device__ __forceinline__ uint32_t pm1_pair(uint32_t w) {
-  return ((w << (15 - Q)) & 0x80008000u) | 0x3C003C00u;
-}
-
-// Same with a run-time pair index.
-__device__ __forceinline__ uint32_t pm1_pair_rt(uint32_t w, int q) {
-  return ((w << (15 - q)) & 0x80008000u) | 0x3C003C00u;
+// fp16 pair (+-1, +-1) for group g of word w: shift bits (g, g+16) to the two
+// fp16 sign positions (15, 31) and OR them into the pair (1.0, 1.0).
+__device__ __forceinline__ uint32_t pm1_pair_rt(uint32_t w, int g) {
+  return ((w << (15 - g)) & 0x80008000u) | 0x3C003C00u;
 }
 
 // fp16 pair (+-s0, +-s1): flip the sign bits of the scale pair where the
 // packed bits are set.  Exact for any fp16 scale.
-__device__ __forceinline__ uint32_t signed_scale_pair_rt(uint32_t w, int q, uint32_t scale_pair) {
-  return ((w << (15 - q)) & 0x80008000u) ^ scale_pair;
+__device__ __forceinline__ uint32_t signed_scale_pair_rt(uint32_t w, int g, uint32_t scale_pair) {
+  return ((w << (15 - g)) & 0x80008000u) ^ scale_pair;
+}
+
+// 1-D bulk copy global -> shared, completion counted in bytes on `bar`.
+// Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ---------------------------------------------------------------- warp MMA

@@ -26,6 +26,7 @@ struct DecodeArgs {
   int batch;               // 1..16
   int kchunk;              // K elements per cluster rank (multiple of 256)
   int weights_early;       // may read packed/kscale/rowscale before the PDL wait
+  int* status;             // device status word (DBF_ERR_TIMEOUT on a lost wait)
 };
 
 // One sign-product GEMM of the prefill path (same formula, tcgen05).
@@ -64,7 +65,7 @@ dbf_status launch_reconstruct(const uint32_t* packedA, const uint32_t* packedB, 
                               const __half* b, int64_t n, int64_t k, int64_t m_in, void* W, bool out_f32,
                               const DeviceInfo& dev, cudaStream_t stream);
 
-inline int64_t words_per_row(int64_t cols) { return cols <= 0 ? 0 : ((cols + 127) / 128) * 4; }
+inline int64_t words_per_row(int64_t cols) { return cols <= 0 ? 0 : ((cols + 255) / 256) * 8; }
 
 // Plain launch that reports this launch's own error (not a pending one).
 template <typename... KArgs, typename... Args>

@@ -2,9 +2,10 @@
 //
 // The pages store A and B as matrices of +-1 elements ("Addition is almost all
 // you need", sciencestack.ai Figure 1; gist.science section 2.1).  One warp
-// builds one 32-bit word: lane p reads the element that the layout puts at bit
-// p (element 2(p%16) + p/16 of the 32-element group) and a warp ballot of
-// "value < 0" is the word.  Rows are padded to 128 bits with zero bits.
+// builds one 32-bit word: word p of a 256-column block holds the column pair
+// (16g + 2p, 16g + 2p + 1) of every group g at bits (g, g+16), so lane b reads
+// column 16(b%16) + 2p + b/16 of the block and a warp ballot of "value < 0" is
+// the word.  Rows are padded to whole blocks with zero bits.
 // Not a hot path (weights are packed once).
 #include <algorithm>
 
@@ -24,11 +25,12 @@ __global__ void dbf_pack_kernel(const T* __restrict__ src, int64_t rows, int64_t
   const int lane = threadIdx.x & 31;
   const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int elem = 2 * (lane & 15) + (lane >> 4);  // element whose sign is bit `lane`
+  const int lane_col = 16 * (lane & 15) + (lane >> 4);  // column (within its block, for pair 0) of bit `lane`
   const int64_t total = rows * wpr;
   for (int64_t word = warp_id; word < total; word += nwarps) {
     const int64_t r = word / wpr;
-    const int64_t col = (word - r * wpr) * 32 + elem;
+    const int64_t wi = word - r * wpr;
+    const int64_t col = (wi >> 3) * 256 + 2 * (wi & 7) + lane_col;
     const bool neg = col < cols && is_negative(src[r * cols + col]);
     const uint32_t bits = __ballot_sync(0xffffffffu, neg);
     if (lane == 0) packed[word] = bits;

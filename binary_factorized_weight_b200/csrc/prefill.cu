@@ -103,42 +103,64 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     // ------------------------------------------------ sign expansion
+    // Row r's packed row is a sequence of 8-word blocks of 256 columns; K step
+    // kt covers groups 4*(kt%4) .. 4*(kt%4)+3 of block kt/4.  Group g's 16
+    // columns come from bit pair (g, g+16) of the block's 8 words.
     const int r = m0 + tid;
     const bool rok = r < p.M;
-    const uint2* wrow = reinterpret_cast<const uint2*>(p.packed + (rok ? static_cast<int64_t>(r) * p.wpr : 0));
-    uint2 wnext = make_uint2(0u, 0u);
-    if (p.weights_early && rok) wnext = __ldg(wrow);
+    const uint4* wrow = reinterpret_cast<const uint4*>(p.packed + (rok ? static_cast<int64_t>(r) * p.wpr : 0));
+    uint4 nxt0 = make_uint4(0u, 0u, 0u, 0u), nxt1 = nxt0;
+    if (p.weights_early && rok) {
+      nxt0 = __ldg(wrow);
+      nxt1 = __ldg(wrow + 1);
+    }
     pdl_wait();
-    if (!p.weights_early && rok) wnext = __ldg(wrow);
+    if (!p.weights_early && rok) {
+      nxt0 = __ldg(wrow);
+      nxt1 = __ldg(wrow + 1);
+    }
+    uint32_t w[8];
     bool ok = true;
     const int swz = tid & 7;
     for (int kt = 0; kt < KT; ++kt) {
       const int s = kt % S;
       const uint32_t use = static_cast<uint32_t>(kt / S);
-      const uint2 wcur = wnext;
-      if (kt + 1 < KT && rok) wnext = __ldg(wrow + kt + 1);
+      if ((kt & 3) == 0) {
+        w[0] = nxt0.x; w[1] = nxt0.y; w[2] = nxt0.z; w[3] = nxt0.w;
+        w[4] = nxt1.x; w[5] = nxt1.y; w[6] = nxt1.z; w[7] = nxt1.w;
+        const int nb = (kt >> 2) + 1;  // next block
+        if (rok && nb * 4 < KT) {
+          nxt0 = __ldg(wrow + 2 * nb);
+          nxt1 = __ldg(wrow + 2 * nb + 1);
+        }
+      }
       if (kt >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) {
         ok = false;
         break;
       }
       uint8_t* dst = a_st + s * kABytes + (tid >> 3) * 1024 + swz * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t wsel = (j < 4) ? wcur.x : wcur.y;
-        uint32_t h[4];
+      for (int i = 0; i < 4; ++i) {
+        const int g = 4 * (kt & 3) + i;  // group inside the block
+        uint32_t h[8];
         if constexpr (KSCALE) {
-          const uint4 sc = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 8 * j));
-          h[0] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 0, sc.x);
-          h[1] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 1, sc.y);
-          h[2] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 2, sc.z);
-          h[3] = signed_scale_pair_rt(wsel, 4 * (j & 3) + 3, sc.w);
+          const uint4* sc = reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 16 * i);
+          const uint4 s0 = __ldg(sc), s1 = __ldg(sc + 1);
+          h[0] = signed_scale_pair_rt(w[0], g, s0.x);
+          h[1] = signed_scale_pair_rt(w[1], g, s0.y);
+          h[2] = signed_scale_pair_rt(w[2], g, s0.z);
+          h[3] = signed_scale_pair_rt(w[3], g, s0.w);
+          h[4] = signed_scale_pair_rt(w[4], g, s1.x);
+          h[5] = signed_scale_pair_rt(w[5], g, s1.y);
+          h[6] = signed_scale_pair_rt(w[6], g, s1.z);
+          h[7] = signed_scale_pair_rt(w[7], g, s1.w);
         } else {
-          h[0] = pm1_pair_rt(wsel, 4 * (j & 3) + 0);
-          h[1] = pm1_pair_rt(wsel, 4 * (j & 3) + 1);
-          h[2] = pm1_pair_rt(wsel, 4 * (j & 3) + 2);
-          h[3] = pm1_pair_rt(wsel, 4 * (j & 3) + 3);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) h[q] = pm1_pair_rt(w[q], g);
         }
-        *reinterpret_cast<uint4*>(dst + ((j ^ swz) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        // columns 16i..16i+7 -> 16-byte chunk 2i, 16i+8..16i+15 -> chunk 2i+1 (128B swizzle)
+        *reinterpret_cast<uint4*>(dst + (((2 * i) ^ swz) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(dst + (((2 * i + 1) ^ swz) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
       }
       fence_proxy_async_smem();
       mbar_arrive(&full_a[s]);

@@ -4,9 +4,11 @@
 //   W[i][j] = a_i * b_j * sum_l A[i][l] * mid_l * B[l][j]
 //
 // Used to check a factorisation against the dense weight it stands for; not a
-// hot path.  A 64x64 tile of W per CTA, 256 threads with 4x4 outputs each, the
-// middle dimension walked one packed word (32 values) at a time with the sign
-// words staged in shared memory.  fp32 accumulation of +-mid_l.
+// hot path.  A 64x64 tile of W per CTA, 256 threads with 4x4 outputs each; the
+// middle dimension is walked one packed block (256 values of l) at a time with
+// A's block words for the tile's 64 rows and B's block words for 256 rows l
+// (the columns j0..j0+63 of those rows) staged in shared memory.  fp32
+// accumulation of +-mid_l.
 #include "dbf_device.cuh"
 #include "dbf_internal.h"
 
@@ -22,40 +24,38 @@ __global__ void __launch_bounds__(256) dbf_reconstruct_kernel(const uint32_t* __
                                                               const __half* __restrict__ mid,
                                                               const __half* __restrict__ b, int n, int k, int m_in,
                                                               int64_t wprA, int64_t wprB, void* W) {
-  __shared__ uint32_t a_words[kTile];     // rows i0.., word of l-chunk
-  __shared__ uint32_t b_words[32][2];     // rows l.., words covering j0..j0+63
-  __shared__ float mid_s[32];
+  __shared__ uint32_t a_words[kTile][8];   // rows i0.., the 8 words of the l-block
+  __shared__ uint32_t b_words[256][9];     // rows l of the block, B's 8 words of block j0/256 (+1 pad)
+  __shared__ float mid_s[256];
 
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
+  const int64_t jblock_word = static_cast<int64_t>(j0 / 256) * 8;
   float acc[4][4] = {};
 
-  for (int lc = 0; lc < k; lc += 32) {
-    if (tid < kTile) {
-      const int i = i0 + tid;
-      a_words[tid] = i < n ? packedA[static_cast<int64_t>(i) * wprA + (lc >> 5)] : 0u;
-    } else if (tid < kTile + 64) {
-      const int t = tid - kTile;
-      const int l = lc + (t >> 1);
-      const int64_t word = (j0 >> 5) + (t & 1);
-      b_words[t >> 1][t & 1] = (l < k && word < wprB) ? packedB[static_cast<int64_t>(l) * wprB + word] : 0u;
-    } else if (tid < kTile + 64 + 32) {
-      const int t = tid - kTile - 64;
-      mid_s[t] = (lc + t < k) ? __half2float(mid[lc + t]) : 0.f;
+  for (int lb = 0; lb < k; lb += 256) {
+    for (int t = tid; t < kTile * 8; t += 256) {
+      const int i = i0 + (t >> 3);
+      a_words[t >> 3][t & 7] = i < n ? packedA[static_cast<int64_t>(i) * wprA + lb / 32 + (t & 7)] : 0u;
     }
+    for (int t = tid; t < 256 * 8; t += 256) {
+      const int l = lb + (t >> 3);
+      b_words[t >> 3][t & 7] = l < k ? packedB[static_cast<int64_t>(l) * wprB + jblock_word + (t & 7)] : 0u;
+    }
+    mid_s[tid] = (lb + tid < k) ? __half2float(mid[lb + tid]) : 0.f;
     __syncthreads();
-#pragma unroll 4
-    for (int e = 0; e < 32; ++e) {
-      const int bit = packed_bit_of(e);
+    const int lmax = min(256, k - lb);
+    for (int e = 0; e < lmax; ++e) {
+      const int aw = packed_word_in_block(e), abit = packed_bit_in_block(e);
       const float m = mid_s[e];
       float sa[4], sb[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) sa[r] = ((a_words[ty * 4 + r] >> bit) & 1u) ? -m : m;
+      for (int r = 0; r < 4; ++r) sa[r] = ((a_words[ty * 4 + r][aw] >> abit) & 1u) ? -m : m;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int col = tx * 4 + q;
-        sb[q] = ((b_words[e][col >> 5] >> packed_bit_of(col & 31)) & 1u) ? -1.f : 1.f;
+        const int jc = (j0 + tx * 4 + q) & 255;  // column of B within its block
+        sb[q] = ((b_words[e][packed_word_in_block(jc)] >> packed_bit_in_block(jc)) & 1u) ? -1.f : 1.f;
       }
 #pragma unroll
       for (int r = 0; r < 4; ++r)

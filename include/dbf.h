@@ -34,13 +34,15 @@
  * Packed sign layout (the pages only say the factors are binary sign
  * matrices; this bit layout is the library's own choice):
  *  - A rows x cols sign matrix is stored row after row.  Each row occupies
- *    dbf_packed_words_per_row(cols) = ceil(cols/128)*4 little-endian 32-bit
- *    words, so every row starts on a 16-byte boundary.
- *  - Element c of a row is held in word c/32 of that row, at bit
- *    (e/2) + 16*(e%2) with e = c%32: the even elements of the 32-element group
- *    fill bits 0..15 and the odd elements bits 16..31.  Element pair (2q, 2q+1)
- *    therefore sits at bits (q, q+16), the two sign positions of an fp16 pair
- *    after one shift.
+ *    dbf_packed_words_per_row(cols) = ceil(cols/256)*8 little-endian 32-bit
+ *    words: one block of 8 words per 256 columns, so every row starts on a
+ *    32-byte boundary.
+ *  - Inside a block, column e (0..255) belongs to group g = e/16 and pair
+ *    p = (e%16)/2 of that group.  It is held in word p of the block at bit
+ *    g + 16*(e%2).  Word p therefore carries, at bits (g, g+16), the column
+ *    pair (16g + 2p, 16g + 2p + 1) of every group g: one shift and one mask
+ *    turn it into an fp16 pair of signs, and the 16 columns of a group come
+ *    from the same bit pair of the block's 8 words.
  *  - A set bit means -1, a clear bit +1.  Bits past the last column are 0.
  *  - packedA holds A (n rows over k columns); packedB holds B (k rows over
  *    m_in columns): both are packed along the reduction dimension of their
@@ -94,11 +96,11 @@ enum {
   DBF_FWD_DECODE_SHIFT_EXPAND = 1u << 3
 };
 
-/* Words (uint32) in one packed row of `cols` signs: ceil(cols/128)*4.
+/* Words (uint32) in one packed row of `cols` signs: ceil(cols/256)*8.
  * Returns 0 for cols <= 0. */
 DBF_API int64_t dbf_packed_words_per_row(int64_t cols);
 
-/* Words (uint32) of a packed rows x cols sign matrix: rows*ceil(cols/128)*4.
+/* Words (uint32) of a packed rows x cols sign matrix: rows*ceil(cols/256)*8.
  * Returns 0 for rows <= 0 or cols <= 0. */
 DBF_API int64_t dbf_packed_words(int64_t rows, int64_t cols);
 

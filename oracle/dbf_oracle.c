@@ -25,10 +25,12 @@
  * Packed sign layout decoded by oracle_unpack_signs (the pages only say the
  * matrices are binary/sign; the bit layout is this library's own choice):
  *   - a rows x cols sign matrix is stored row after row; each row takes
- *     ceil(cols/128)*4 little-endian 32-bit words (a multiple of 16 bytes);
- *   - element c of a row lives in word c/32; inside that word, element
- *     e = c%32 sits at bit (e/2) + 16*(e%2): even elements fill bits 0..15,
- *     odd elements bits 16..31;
+ *     ceil(cols/256)*8 little-endian 32-bit words (a multiple of 32 bytes),
+ *     one block of 8 words per 256 columns;
+ *   - inside a block, column e (0..255) belongs to group g = e/16 and pair
+ *     p = (e%16)/2 of that group; it is held in word p of the block, at bit
+ *     g + 16*(e%2).  So word p carries pair p of all 16 groups, even columns
+ *     in bits 0..15 and odd columns in bits 16..31;
  *   - a set bit means -1, a clear bit +1; bits past the last column are 0.
  *
  * Parity status of each function (see the test-suite pins in
@@ -53,11 +55,12 @@ int oracle_num_threads(void) {
 #endif
 }
 
-/* Words per packed row: the row is padded to a multiple of 128 bits. */
-int64_t oracle_words_per_row(int64_t cols) { return ((cols + 127) / 128) * 4; }
+/* Words per packed row: the row is padded to a multiple of 256 columns. */
+int64_t oracle_words_per_row(int64_t cols) { return ((cols + 255) / 256) * 8; }
 
-/* Bit position of element e (0..31) inside its 32-bit word. */
-static int bit_of_element(int e) { return (e >> 1) + ((e & 1) << 4); }
+/* Word (within the row) and bit holding column c. */
+static int64_t word_of_column(int64_t c) { return (c / 256) * 8 + (c % 16) / 2; }
+static int bit_of_column(int64_t c) { return (int)((c % 256) / 16) + 16 * (int)(c % 2); }
 
 /*
  * Decode a packed sign matrix into int8 +-1 values (row-major rows x cols).
@@ -69,14 +72,12 @@ int64_t oracle_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, 
   for (int64_t r = 0; r < rows; ++r) {
     const uint32_t* row = packed + r * wpr;
     for (int64_t c = 0; c < cols; ++c) {
-      uint32_t word = row[c / 32];
-      int bit = bit_of_element((int)(c % 32));
-      out[r * cols + c] = ((word >> bit) & 1u) ? (int8_t)-1 : (int8_t)1;
+      uint32_t word = row[word_of_column(c)];
+      out[r * cols + c] = ((word >> bit_of_column(c)) & 1u) ? (int8_t)-1 : (int8_t)1;
     }
     for (int64_t c = cols; c < wpr * 32; ++c) {
-      uint32_t word = row[c / 32];
-      int bit = bit_of_element((int)(c % 32));
-      bad_padding += (word >> bit) & 1u;
+      uint32_t word = row[word_of_column(c)];
+      bad_padding += (word >> bit_of_column(c)) & 1u;
     }
   }
   return bad_padding;
@@ -92,7 +93,7 @@ void oracle_pack_signs(const int8_t* signs, int64_t rows, int64_t cols, uint32_t
   for (int64_t r = 0; r < rows; ++r) {
     for (int64_t c = 0; c < cols; ++c) {
       if (signs[r * cols + c] < 0) {
-        packed[r * wpr + c / 32] |= 1u << bit_of_element((int)(c % 32));
+        packed[r * wpr + word_of_column(c)] |= 1u << bit_of_column(c);
       }
     }
   }

@@ -45,9 +45,10 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_packed_words(lib):
-    assert dbf.dbf_packed_words_per_row(1) == 4
-    assert dbf.dbf_packed_words_per_row(128) == 4
-    assert dbf.dbf_packed_words_per_row(129) == 8
+    assert dbf.dbf_packed_words_per_row(1) == 8
+    assert dbf.dbf_packed_words_per_row(256) == 8
+    assert dbf.dbf_packed_words_per_row(257) == 16
+    assert dbf.dbf_packed_words_per_row(832) == 32
     assert dbf.dbf_packed_words_per_row(4096) == 128
     assert dbf.dbf_packed_words(4096, 2048) == 4096 * 64
     assert dbf.dbf_packed_words(0, 64) == 0

@@ -27,7 +27,10 @@ MUTANTS = {
     "dropped_last_term": ("for (int64_t l = 0; l < k; ++l) acc += (double)Ai[l]",
                           "for (int64_t l = 0; l + 1 < k; ++l) acc += (double)Ai[l]"),
     "mid_indexed_by_row": ("vbuf[l] = mid[l] * acc;", "vbuf[l] = mid[l % (k > 1 ? k - 1 : 1)] * acc;"),
-    "natural_bit_layout": ("return (e >> 1) + ((e & 1) << 4);", "return e;"),
+    "natural_bit_layout": ("static int bit_of_column(int64_t c) { return (int)((c % 256) / 16) + 16 * (int)(c % 2); }",
+                           "static int bit_of_column(int64_t c) { return (int)(c % 32); }"),
+    "words_per_32_columns": ("static int64_t word_of_column(int64_t c) { return (c / 256) * 8 + (c % 16) / 2; }",
+                             "static int64_t word_of_column(int64_t c) { return c / 32; }"),
     "dense_drops_b": ("Wi[j] += left * ((double)Bl[j] * b[j]);", "Wi[j] += left * ((double)Bl[j]);"),
     "dense_transposed_B": ("Wi[j] += left * ((double)Bl[j] * b[j]);",
                            "Wi[j] += left * ((double)B[(j % k) * m_in + (l % m_in)] * b[j]);"),
@@ -47,6 +50,7 @@ PIN_CHECKS = [
     lambda o: pins.test_bits_per_weight_closed_form(o, 4096, 2048, 4096, 1.0),
     lambda o: pins.test_layout_table(o),
     lambda o: pins.test_layout_round_trip_and_padding(o, 3, 128),
+    lambda o: pins.test_layout_hand_words(o),
 ]
 
 

@@ -234,13 +234,14 @@ def test_orientation_is_not_transposed(oracle_mod):
 @pytest.mark.parametrize(
     "n,k,m_in,expect",
     [(4096, 2048, 4096, 1.0), (4096, 4096, 4096, 2.0), (14336, 4736, 4096, 4736 * 18432 / (14336 * 4096)),
-     (256, 128, 256, 1.0)],
+     (256, 256, 256, 2.0), (256, 128, 256, 1.0)],
 )
 def test_bits_per_weight_closed_form(oracle_mod, n, k, m_in, expect):
     assert oracle_mod.bits_per_weight(n, k, m_in) == pytest.approx(expect, rel=1e-15)
-    # packed sign storage: rows are 128-aligned here, so bits = k*n + k*m_in exactly
-    words = n * oracle_mod.words_per_row(k) + k * oracle_mod.words_per_row(m_in)
-    assert words * 32 / (n * m_in) == pytest.approx(expect, rel=1e-15)
+    # packed sign storage: with k and m_in multiples of 256 there is no padding, so bits = k*n + k*m_in
+    if k % 256 == 0 and m_in % 256 == 0:
+        words = n * oracle_mod.words_per_row(k) + k * oracle_mod.words_per_row(m_in)
+        assert words * 32 / (n * m_in) == pytest.approx(expect, rel=1e-15)
     assert oracle_mod.scale_bits_per_weight(n, k, m_in) == pytest.approx(16 * (n + k + m_in) / (n * m_in))
 
 
@@ -256,42 +257,65 @@ def test_bits_per_weight_rounding_rule():
 
 
 # ---------------------------------------------------------------- packed layout
+def _layout_table():
+    rows = []
+    from conftest import GOLDEN
+    import os
+
+    with open(os.path.join(GOLDEN, "packed_layout_bits.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(tuple(int(v) for v in line.split()))
+    return rows
+
+
 def test_layout_table(oracle_mod):
-    table = read_golden("packed_layout_bits.txt")
-    for e_str, (bit,) in table.items():
-        e = int(e_str)
-        signs = np.ones((1, 32), dtype=np.int8)
-        signs[0, e] = -1
+    for col, word, bit in _layout_table():
+        cols = 768
+        wpr = (cols + 255) // 256 * 8
+        signs = np.ones((1, cols), dtype=np.int8)
+        signs[0, col] = -1
         packed = oracle_mod.pack_signs(signs)
-        assert packed.tolist() == [1 << int(bit), 0, 0, 0]
-        back, bad = oracle_mod.unpack_signs(np.array([1 << int(bit), 0, 0, 0], dtype=np.uint32), 1, 32)
+        expect = np.zeros(wpr, dtype=np.uint32)
+        expect[word] = np.uint32(1 << bit)
+        assert np.array_equal(packed, expect), (col, word, bit)
+        back, bad = oracle_mod.unpack_signs(expect, 1, cols)
         assert bad == 0 and np.array_equal(back, signs)
 
 
 def test_layout_hand_words(oracle_mod):
-    # 0x0000FFFF: bits 0..15 set -> even elements are -1, odd are +1
-    back, bad = oracle_mod.unpack_signs(np.array([0x0000FFFF, 0, 0, 0], dtype=np.uint32), 1, 32)
-    assert bad == 0
-    assert back[0].tolist() == [-1 if e % 2 == 0 else 1 for e in range(32)]
-    # second word of a row holds elements 32..63; rows are 4 words apart for cols <= 128
+    # word 0 = 0x0000FFFF: bits 0..15 are pair 0, even column, of groups 0..15 -> columns 0, 16, ..., 240
     packed = np.zeros(8, dtype=np.uint32)
-    packed[1] = 1 << 16  # element 33
-    packed[4 + 3] = 1 << 31  # row 1, element 127
-    back, bad = oracle_mod.unpack_signs(packed, 2, 128)
+    packed[0] = 0x0000FFFF
+    back, bad = oracle_mod.unpack_signs(packed, 1, 256)
     assert bad == 0
-    assert [int(i) for i in np.nonzero(back[0] < 0)[0]] == [33]
-    assert [int(i) for i in np.nonzero(back[1] < 0)[0]] == [127]
+    assert [int(i) for i in np.nonzero(back[0] < 0)[0]] == list(range(0, 256, 16))
+    # word 3 = 0xFFFF0000: bits 16..31 are pair 3, odd column -> columns 16g + 7
+    packed[:] = 0
+    packed[3] = 0xFFFF0000
+    back, _ = oracle_mod.unpack_signs(packed, 1, 256)
+    assert [int(i) for i in np.nonzero(back[0] < 0)[0]] == [16 * g + 7 for g in range(16)]
+    # rows are 8 words apart for cols <= 256; second block of a row starts at word 8
+    packed = np.zeros(32, dtype=np.uint32)
+    packed[8] = 1 << 16  # row 0, column 257
+    packed[16 + 15] = 1 << 31  # row 1, column 511
+    back, bad = oracle_mod.unpack_signs(packed, 2, 512)
+    assert bad == 0
+    assert [int(i) for i in np.nonzero(back[0] < 0)[0]] == [257]
+    assert [int(i) for i in np.nonzero(back[1] < 0)[0]] == [511]
 
 
-@pytest.mark.parametrize("rows,cols", [(1, 64), (3, 128), (5, 192), (17, 320), (2, 1000)])
+@pytest.mark.parametrize("rows,cols", [(1, 64), (3, 128), (5, 192), (17, 320), (2, 1000), (4, 832)])
 def test_layout_round_trip_and_padding(oracle_mod, rows, cols):
     rng = np.random.default_rng(rows * cols)
     s = gen.sign_matrix(rng, rows, cols)
     packed = oracle_mod.pack_signs(s)
-    assert packed.size == rows * ((cols + 127) // 128) * 4
+    wpr = ((cols + 255) // 256) * 8
+    assert packed.size == rows * wpr
     back, bad = oracle_mod.unpack_signs(packed, rows, cols)
     assert bad == 0 and np.array_equal(back, s)
-    if cols % 128:
+    if cols % 256:
         corrupt = packed.copy()
-        corrupt[((cols + 127) // 128) * 4 - 1] |= np.uint32(1 << 31)  # last padding bit of row 0
+        corrupt[wpr - 1] |= np.uint32(1 << 31)  # group 15, pair 7, odd: column 255 of the last block
         assert oracle_mod.unpack_signs(corrupt, rows, cols)[1] == 1
