@@ -29,7 +29,7 @@ __all__ = [
     "library_path", "load_library",
     "dbf_packed_words_per_row", "dbf_packed_words", "dbf_pack_signs",
     "dbf_forward_workspace_bytes", "dbf_new_workspace", "dbf_forward",
-    "dbf_reconstruct_dense", "dbf_workspace_status", "dbf_status_string",
+    "dbf_reconstruct_dense", "dbf_workspace_status", "dbf_status_string", "dbf_forward_noalloc",
 ]
 
 DBF_I8, DBF_F16, DBF_F32 = 0, 1, 2
@@ -51,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "dbf_forward",
     "dbf_reconstruct_dense",
     "dbf_workspace_status",
+    "dbf_forward_noalloc",
     "dbf_status_string",
 )
 
@@ -92,6 +93,8 @@ def load_library():
     lib.dbf_reconstruct_dense.restype = i32
     lib.dbf_workspace_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
     lib.dbf_workspace_status.restype = i32
+    lib.dbf_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, u32, vp]
+    lib.dbf_forward_noalloc.restype = i32
     lib.dbf_status_string.argtypes = [i32]
     lib.dbf_status_string.restype = ctypes.c_char_p
     _LIB = lib
@@ -182,6 +185,25 @@ def dbf_forward(x: torch.Tensor, packedA: torch.Tensor, packedB: torch.Tensor, a
     _check("dbf_forward", load_library().dbf_forward(
         _ptr(x), _ptr(packedA), _ptr(packedB), _ptr(a), _ptr(m), _ptr(b), int(n), int(k), int(m_in), int(batch),
         _ptr(y), y_code, _ptr(workspace), workspace.numel() * workspace.element_size(), int(flags), _stream(stream)))
+    return y
+
+
+def dbf_forward_noalloc(x: torch.Tensor, packedA: torch.Tensor, packedB: torch.Tensor, a: torch.Tensor,
+                        m: torch.Tensor, b: torch.Tensor, n: int, k: int, m_in: int, y: Optional[torch.Tensor] = None,
+                        y_dtype: torch.dtype = torch.float16, flags: int = 0, stream=None) -> torch.Tensor:
+    """dbf_forward without a workspace, for callers that cannot allocate device memory.
+
+    The library's own 2 MiB buffer stands in for the workspace (limit: 256 + batch*k*2
+    bytes); every call shares it, so calls that overlap on the GPU race.  The first call
+    on a device looks the buffer up; make it before any stream capture."""
+    if x.dtype != torch.float16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp16 batch x m_in tensor")
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, n), dtype=y_dtype, device=x.device)
+    _check("dbf_forward_noalloc", load_library().dbf_forward_noalloc(
+        _ptr(x), _ptr(packedA), _ptr(packedB), _ptr(a), _ptr(m), _ptr(b), int(n), int(k), int(m_in), int(batch),
+        _ptr(y), _dtype_code(y.dtype), int(flags), _stream(stream)))
     return y
 
 

@@ -178,6 +178,32 @@ DBF_API dbf_status dbf_reconstruct_dense(const uint32_t* packedA, const uint32_t
  */
 DBF_API dbf_status dbf_workspace_status(const void* workspace, struct CUstream_st* stream, int32_t* device_status);
 
+/*
+ * dbf_forward for callers that cannot allocate device memory.  (The pages have
+ * no counterpart: this concerns who provides the scratch buffer, not the
+ * method.)  Some callers have no allocator to hand: a plugin inside a host
+ * application that owns all device memory and offers its extensions none, or
+ * a latency-critical thread that must not call cudaMalloc (which can block
+ * and synchronise the device).  This call takes the same arguments as
+ * dbf_forward minus the workspace and uses instead a 2 MiB buffer that lives
+ * in the library (a static __device__ array, held by every GPU that loads the
+ * library until the process exits).  It allocates and frees nothing.
+ *   Limit: dbf_forward_workspace_bytes(n, k, m_in, batch) <= 2 MiB, i.e.
+ *   256 + batch*k*2 bytes (e.g. batch 16 with k up to 65528, or batch 256 with
+ *   k up to 4095); larger sizes return DBF_ERR_WORKSPACE.
+ *   The first call on each device looks up the buffer's device address with
+ *   that device current; make that first call before any stream capture.
+ *   Each call clears the buffer's status word (cudaMemsetAsync on `stream`)
+ *   before its kernels; the buffer keeps the last call's other contents.
+ *   All calls share the one buffer: calls whose work overlaps on the GPU
+ *   (other streams, other host threads) race on it and must be serialised by
+ *   the caller.  Argument checks are those of dbf_forward and run first.
+ */
+DBF_API dbf_status dbf_forward_noalloc(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB,
+                                       const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n,
+                                       int64_t k, int64_t m_in, int64_t batch, void* y, dbf_dtype y_t,
+                                       uint32_t flags, struct CUstream_st* stream);
+
 /* Static, NUL-terminated description of a status code. */
 DBF_API const char* dbf_status_string(dbf_status status);
 

@@ -122,6 +122,18 @@ def test_reconstruct_validation(lib):
     assert lib.dbf_reconstruct_dense(P, P, P, P, P, 256, 128, 256, MIS, 2, None) == MISALIGNED
 
 
+def test_noalloc_validation(lib):
+    # same argument checks as dbf_forward, then the 2 MiB limit of its own buffer
+    def call(x=P, n=256, k=128, m_in=256, batch=4, y_t=1, flags=0):
+        return lib.dbf_forward_noalloc(x, P, P, P, P, P, n, k, m_in, batch, P, y_t, flags, None)
+
+    assert call(x=None) == INVALID
+    assert call(k=96) == SHAPE
+    assert call(x=MIS) == MISALIGNED
+    assert call(flags=1 << 9) == INVALID
+    assert call(k=16384, batch=64) == WORKSPACE  # 256 + 64*16384*2 bytes > 2 MiB
+
+
 def test_workspace_status_validation(lib):
     out = ctypes.c_int32()
     assert lib.dbf_workspace_status(None, None, ctypes.byref(out)) == INVALID
