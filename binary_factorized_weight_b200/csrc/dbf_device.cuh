@@ -57,6 +57,15 @@ __device__ __forceinline__ uint32_t signed_scale_pair_rt(uint32_t w, int g, uint
   return ((w << (15 - g)) & 0x80008000u) ^ scale_pair;
 }
 
+// Streaming 16-byte load that does not allocate in L1 (weights are read once).
+__device__ __forceinline__ uint4 ldg_stream_u4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // 1-D bulk copy global -> shared, completion counted in bytes on `bar`.
 // Addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {

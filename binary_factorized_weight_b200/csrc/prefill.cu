@@ -17,16 +17,20 @@
 // The kernel is persistent: one CTA per SM walks the tiles tile = blockIdx.x,
 // + gridDim.x, ...; the shared-memory ring runs on across tiles, and two TMEM
 // accumulators let the epilogue of one tile overlap the main loop of the next.
-// Roles (320 threads):
-//   warps 0-3  sign expansion: thread r turns row r's packed bits of a K step
-//              into 64 fp16 values (+-1, or +-b_j with b folded in by flipping
-//              the scale's sign bit: exact) stored as one 128-byte row of a
-//              128B-swizzled K-major tile;
-//   warp 4     TMA producer of the activation tile (K-major, 128B swizzle,
-//              tokens past the batch read as zero);
-//   warp 5     TMEM allocation and the single-thread tcgen05.mma issue loop;
-//   warps 6-9  epilogue: TMEM -> registers -> row scale -> global stores
-//              (warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31).
+// Roles (448 threads):
+//   warps 0-7   sign expansion: thread t owns weight row t%128 and word half
+//               t/128 of each 8-word block, i.e. pairs 4h..4h+3 of every
+//               16-column group.  Per K step it turns 32 sign bits into 32
+//               fp16 values (+-1, or +-b_j with b folded in by flipping the
+//               scale's sign bit: exact) and stores four 16-byte chunks of the
+//               row of a 128B-swizzled K-major tile.  Weight blocks are fetched
+//               two blocks ahead and b one K step ahead;
+//   warp 8      TMA producer of the activation tile (K-major, 128B swizzle,
+//               tokens past the batch read as zero);
+//   warp 9      TMEM allocation and the single-thread tcgen05.mma issue loop;
+//   warps 10-13 epilogue: TMEM -> registers -> row scale -> a 32x32 transpose
+//               in shared memory -> 16-byte global stores (warp w reads TMEM
+//               lanes 32*(w%4) .. 32*(w%4)+31).
 // Stage hand-off is through mbarriers; every wait is bounded and an expired
 // wait records DBF_ERR_TIMEOUT in the workspace status word, raises a CTA-wide
 // abort flag and lets all roles fall through to the teardown, which frees TMEM
@@ -36,6 +40,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "dbf_device.cuh"
 #include "dbf_internal.h"
@@ -45,14 +50,20 @@ namespace {
 
 constexpr int kBM = 128;  // weight rows per tile (TMEM lanes)
 constexpr int kBK = 64;   // K per pipeline stage: one 128-byte swizzle row of fp16
-constexpr int kThreads = 320;
+constexpr int kExpThreads = 256;
+constexpr int kThreads = kExpThreads + 32 + 32 + 128;
+constexpr int kWarpTma = kExpThreads / 32;
+constexpr int kWarpMma = kWarpTma + 1;
+constexpr int kWarpEpi0 = kWarpMma + 1;
 constexpr int kABytes = kBM * kBK * 2;
+constexpr int kEpiStageBytes = 32 * 32 * 4;  // one warp's 32 tokens x 32 rows (fp32 worst case)
 
 template <int NTILE>
 struct Cfg {
   static constexpr int kStages = NTILE == 256 ? 4 : 6;
   static constexpr int kBBytes = NTILE * kBK * 2;
-  static constexpr int kBarOffset = kStages * (kABytes + kBBytes);
+  static constexpr int kEpiOffset = kStages * (kABytes + kBBytes);
+  static constexpr int kBarOffset = kEpiOffset + 4 * kEpiStageBytes;
   // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done
   static constexpr int kNumBars = 3 * kStages + 5;
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;  // + tmem slot/abort + align slack
@@ -68,6 +79,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_st = smem;
   uint8_t* b_st = smem + S * kABytes;
+  uint8_t* epi_st = smem + C::kEpiOffset;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* full_a = bars;
   uint64_t* full_b = bars + S;
@@ -86,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full_a[i], 128);
+      mbar_init(&full_a[i], kExpThreads);
       mbar_init(&full_b[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -98,8 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) prefetch_tmap(&act_map);
-  if (warp == 5) {
+  if (warp == kWarpTma && lane == 0) prefetch_tmap(&act_map);
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
@@ -108,79 +120,93 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp < kWarpTma) {
     // ------------------------------------------------ sign expansion
     // Row r's packed row is a sequence of 8-word blocks of 256 columns; K step
-    // kt covers groups 4*(kt%4) .. 4*(kt%4)+3 of block kt/4.  Group g's 16
-    // columns come from bit pair (g, g+16) of the block's 8 words.  The next
-    // block (possibly the first block of this CTA's next tile) is always in
-    // flight while the current one is expanded.
+    // kt covers groups 4*(kt%4) .. 4*(kt%4)+3 of block kt/4, and group g's 16
+    // columns come from bit pair (g, g+16) of the block's 8 words.  This thread
+    // holds words 4h..4h+3 (column pairs 4h..4h+3 of every group).
+    const int r_local = tid & (kBM - 1);
+    const int h = tid >> 7;
     const int nblk = (KT + 3) / 4;
-    auto block_ptr = [&](int tile, int blk) -> const uint4* {
-      const int r = (tile % m_tiles) * kBM + tid;
-      if (tile >= num_tiles || r >= p.M) return nullptr;
-      return reinterpret_cast<const uint4*>(p.packed + static_cast<int64_t>(r) * p.wpr) + 2 * blk;
-    };
-    int tile = blockIdx.x;
-    uint4 nxt0 = make_uint4(0u, 0u, 0u, 0u), nxt1 = nxt0;
-    auto fetch = [&](const uint4* q) {
-      if (q) {
-        nxt0 = __ldg(q);
-        nxt1 = __ldg(q + 1);
-      } else {
-        nxt0 = nxt1 = make_uint4(0u, 0u, 0u, 0u);
+    // block sequence of this CTA: (tile, blk) with blk fastest
+    int f_tile = blockIdx.x, f_blk = 0;
+    auto fetch_next = [&]() -> uint4 {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (f_tile < num_tiles) {
+        const int r = (f_tile % m_tiles) * kBM + r_local;
+        if (r < p.M) v = ldg_stream_u4(p.packed + static_cast<int64_t>(r) * p.wpr + 8 * f_blk + 4 * h);
+        if (++f_blk == nblk) {
+          f_blk = 0;
+          f_tile += gridDim.x;
+        }
       }
+      return v;
     };
-    if (p.weights_early) fetch(block_ptr(tile, 0));
+    auto fetch_scale = [&](int kt, uint4 (&sc)[4]) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        sc[i] = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 16 * i + 8 * h));
+    };
+    uint4 w_n1, w_n2, wcur = make_uint4(0u, 0u, 0u, 0u);
+    uint4 sc_next[4];
+    if (p.weights_early) {
+      w_n1 = fetch_next();
+      w_n2 = fetch_next();
+      if constexpr (KSCALE) fetch_scale(0, sc_next);
+    }
     pdl_wait();
-    if (!p.weights_early) fetch(block_ptr(tile, 0));
-    uint32_t w[8];
+    if (!p.weights_early) {
+      w_n1 = fetch_next();
+      w_n2 = fetch_next();
+      if constexpr (KSCALE) fetch_scale(0, sc_next);
+    }
     bool ok = true;
-    const int swz = tid & 7;
+    const int swz = r_local & 7;
     uint32_t it = 0;
-    for (; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       for (int kt = 0; kt < KT; ++kt, ++it) {
         const int s = static_cast<int>(it % S);
         const uint32_t use = it / S;
         if ((kt & 3) == 0) {
-          w[0] = nxt0.x; w[1] = nxt0.y; w[2] = nxt0.z; w[3] = nxt0.w;
-          w[4] = nxt1.x; w[5] = nxt1.y; w[6] = nxt1.z; w[7] = nxt1.w;
-          const int nb = (kt >> 2) + 1;
-          fetch(nb < nblk ? block_ptr(tile, nb) : block_ptr(tile + gridDim.x, 0));
+          wcur = w_n1;
+          w_n1 = w_n2;
+          w_n2 = fetch_next();
+        }
+        uint4 sc[4];
+        if constexpr (KSCALE) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sc[i] = sc_next[i];
+          fetch_scale(kt + 1 < KT ? kt + 1 : 0, sc_next);
         }
         if (it >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
-        uint8_t* dst = a_st + s * kABytes + (tid >> 3) * 1024 + swz * 128;
+        uint8_t* dst = a_st + s * kABytes + (r_local >> 3) * 1024 + swz * 128;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int g = 4 * (kt & 3) + i;  // group inside the block
-          uint32_t h[8];
+          uint32_t q[4];
           if constexpr (KSCALE) {
-            const uint4* sc = reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 16 * i);
-            const uint4 s0 = __ldg(sc), s1 = __ldg(sc + 1);
-            h[0] = signed_scale_pair_rt(w[0], g, s0.x);
-            h[1] = signed_scale_pair_rt(w[1], g, s0.y);
-            h[2] = signed_scale_pair_rt(w[2], g, s0.z);
-            h[3] = signed_scale_pair_rt(w[3], g, s0.w);
-            h[4] = signed_scale_pair_rt(w[4], g, s1.x);
-            h[5] = signed_scale_pair_rt(w[5], g, s1.y);
-            h[6] = signed_scale_pair_rt(w[6], g, s1.z);
-            h[7] = signed_scale_pair_rt(w[7], g, s1.w);
+            q[0] = signed_scale_pair_rt(wcur.x, g, sc[i].x);
+            q[1] = signed_scale_pair_rt(wcur.y, g, sc[i].y);
+            q[2] = signed_scale_pair_rt(wcur.z, g, sc[i].z);
+            q[3] = signed_scale_pair_rt(wcur.w, g, sc[i].w);
           } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) h[q] = pm1_pair_rt(w[q], g);
+            q[0] = pm1_pair_rt(wcur.x, g);
+            q[1] = pm1_pair_rt(wcur.y, g);
+            q[2] = pm1_pair_rt(wcur.z, g);
+            q[3] = pm1_pair_rt(wcur.w, g);
           }
-          // columns 16i..16i+7 -> 16-byte chunk 2i, 16i+8..16i+15 -> chunk 2i+1 (128B swizzle)
-          *reinterpret_cast<uint4*>(dst + (((2 * i) ^ swz) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(dst + (((2 * i + 1) ^ swz) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+          // columns 16i + 8h .. 16i + 8h + 7 -> 16-byte chunk 2i + h (128B swizzle)
+          *reinterpret_cast<uint4*>(dst + (((2 * i + h) ^ swz) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(&full_a[s]);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kWarpTma) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       pdl_wait();
@@ -200,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------ MMA issue
     if (lane == 0) {
       pdl_wait();
@@ -239,7 +265,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    using OutT = typename std::conditional<OUT_F32, float, __half>::type;
+    constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
+    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+    OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
+    OutT* out = static_cast<OutT*>(p.out);
+    const bool ld_ok = (p.ld_out % kVec) == 0;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const uint32_t buf = local & 1;
@@ -247,24 +278,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int m0 = (tile % m_tiles) * kBM;
       const int n0 = (tile / m_tiles) * NTILE;
-      const int row = m0 + q * 32 + lane;
+      const int row0 = m0 + q * 32;
+      const int row = row0 + lane;
       const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;
+      const bool rows_full = row0 + 32 <= p.M;
       for (int col = 0; col < NTILE; col += 32) {
         if (n0 + col >= p.batch) break;  // warp-uniform
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * NTILE + static_cast<uint32_t>(col),
                            v);
         tmem_ld_wait();
-        if (row < p.M) {
+        const int tok0 = n0 + col;
+        if (rows_full && ld_ok && tok0 + 32 <= p.batch) {
+          // transpose through shared memory, then 16-byte stores of kVec consecutive rows
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int tok = n0 + col + j;
+            const float val = rs * __uint_as_float(v[j]);
+            if constexpr (OUT_F32) {
+              stg[j * 32 + lane] = val;
+            } else {
+              stg[j * 32 + lane] = __float2half_rn(val);
+            }
+          }
+          __syncwarp();
+          constexpr int kChunksPerTok = 32 / kVec;
+#pragma unroll
+          for (int m = 0; m < 32 * kChunksPerTok / 32; ++m) {
+            const int cidx = lane + 32 * m;
+            const int tk = cidx / kChunksPerTok, rp = cidx % kChunksPerTok;
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + tk * 32 + rp * kVec);
+            *reinterpret_cast<uint4*>(out + static_cast<int64_t>(tok0 + tk) * p.ld_out + row0 + rp * kVec) = val;
+          }
+          __syncwarp();
+        } else if (row < p.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int tok = tok0 + j;
             if (tok < p.batch) {
               const float val = rs * __uint_as_float(v[j]);
               if constexpr (OUT_F32) {
-                static_cast<float*>(p.out)[static_cast<int64_t>(tok) * p.ld_out + row] = val;
+                out[static_cast<int64_t>(tok) * p.ld_out + row] = val;
               } else {
-                static_cast<__half*>(p.out)[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(val);
+                out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(val);
               }
             }
           }
@@ -278,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     // Free TMEM once every MMA this CTA issued has finished (the wait is
     // bounded; TMEM must be released before the CTA exits either way).
