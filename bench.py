@@ -437,6 +437,32 @@ def run_ours(args, shape, batch):
 
 
 # ------------------------------------------------------------------ sweep (all configs, one GPU)
+def dense_fp16_us(torch, shape, batch, device):
+    """Context only (not the product): torch.matmul of x with a dense fp16 W of the
+    same shape, W rotated over copies larger than 4x L2 like the DBF layers."""
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    wbytes = 2 * shape.n * shape.m_in
+    copies = max(2, int(math.ceil(4 * l2 / wbytes)))
+    Ws = [torch.randn(shape.n, shape.m_in, device=device, dtype=torch.float16) for _ in range(copies)]
+    x = torch.randn(batch, shape.m_in, device=device, dtype=torch.float16)
+    y = torch.empty(batch, shape.n, device=device, dtype=torch.float16)
+    for W in Ws[:3]:
+        torch.matmul(x, W.t(), out=y)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for W in Ws:
+            torch.matmul(x, W.t(), out=y)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / copies * 1e3)
+    del Ws
+    torch.cuda.empty_cache()
+    return statistics.median(times)
+
+
 def run_sweep(args):
     import torch
 
@@ -475,11 +501,14 @@ def run_sweep(args):
         us = statistics.median(times)
         gbs = wl.bytes / (us * 1e-6) / 1e9
         tf = layer_flops(shape.n, shape.k, shape.m_in, batch) / (us * 1e-6) / 1e12
+        dense_us = dense_fp16_us(torch, shape, batch, device)
         row = {"layer": shape.name, "n": shape.n, "k": shape.k, "m_in": shape.m_in, "batch": batch,
                "bpw": shape.k * (shape.n + shape.m_in) / (shape.n * shape.m_in), "us": us,
                "us_p10": sorted(times)[0], "us_p90": sorted(times)[-1], "tokens_per_s": batch / (us * 1e-6),
                "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": tf,
-               "tensor_frac": tf / peaks["bf16_tflops"], "copies": wl.copies, "path": wl.path}
+               "tensor_frac": tf / peaks["bf16_tflops"], "copies": wl.copies, "path": wl.path,
+               "context_torch_fp16_dense_us": dense_us,
+               "speedup_vs_dense_fp16": dense_us / us}
         rows.append(row)
         print(json.dumps(row), flush=True)
         del g, wl
