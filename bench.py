@@ -145,6 +145,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside), "window": window}
 
 
+def max_over_ranks(value_ms, world, device=None):
+    """The slowest rank's time (every rank takes part; a no-op on one rank)."""
+    if world <= 1:
+        return float(value_ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, elapsed_ms):
+    """Units all ranks processed per second (weak scaling: every rank does the same work)."""
+    return world * units_per_rank / (elapsed_ms * 1e-3)
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -303,17 +320,13 @@ def run_ours(args, shape, batch):
     torch.cuda.synchronize()
     t_wall1 = time.time()
     barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
 
     ms_per_step = ms / args.steps
     us_per_layer = 1e3 * ms_per_step / wl.copies
-    tokens_per_s = world * batch / (us_per_layer * 1e-6)
+    tokens_per_s = whole_job_rate(batch * wl.copies * args.steps, world, ms)
     hbm_gbs = wl.bytes / (us_per_layer * 1e-6) / 1e9
 
     # ---------------------------------------------------------- end to end: host buffers, copies inside
@@ -346,12 +359,8 @@ def run_ours(args, shape, batch):
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * batch * wl.copies * e2e_steps / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_value = whole_job_rate(batch * wl.copies * e2e_steps, world, e2e_ms)
 
     # output check of the timed configuration (sampled, against the oracle)
     check = None
