@@ -152,6 +152,7 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
       sb.ld_out = k;
       sb.batch = nb;
       sb.weights_early = early ? 1 : 0;
+      sb.peer_rows = static_cast<int>(n);
       sb.status = status;
       st = launch_decode_stage(sb, class_expand, /*out_f32=*/false, dev, stream);
       if (st != DBF_OK) return st;
@@ -168,6 +169,7 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
       sa.ld_out = n;
       sa.batch = nb;
       sa.weights_early = 1;  // stage B releases stage A only after its own wait
+      sa.peer_rows = static_cast<int>(k);
       sa.status = status;
       st = launch_decode_stage(sa, class_expand, out_f32, dev, stream);
       if (st != DBF_OK) return st;

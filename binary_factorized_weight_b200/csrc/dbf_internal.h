@@ -26,6 +26,7 @@ struct DecodeArgs {
   int batch;               // 1..16
   int kchunk;              // K elements per cluster rank (multiple of 256)
   int weights_early;       // may read packed/kscale/rowscale before the PDL wait
+  int peer_rows;           // rows of the forward's other stage (shapes the work split)
   int* status;             // device status word (DBF_ERR_TIMEOUT on a lost wait)
 };
 

@@ -433,37 +433,52 @@ dbf_status launch_rt(const DecodeArgs& a, bool class_expand, bool out_f32, int k
 
 }  // namespace
 
-// Work split of one stage: RT row tiles per CTA (RT*16 rows; the other 4/RT
-// warps of the CTA split K) and ks CTAs per cluster along K.  The choice keeps
-// the activation range a CTA stages (batch x K/ks fp16) inside shared memory,
-// keeps the L2 traffic of restaging activations (one copy per CTA row group)
-// small next to the weight bytes, and aims for one to two CTAs per SM.
+// Work split of one stage: RT*16-row CTAs (RT = 4: 64 rows, one 16-row tile
+// per warp) and ks CTAs per cluster along K.  Measured on B200 over the layer
+// shapes of the workloads at batch 1 and 16, with the weights streamed from HBM:
+//  * a warp's weights should fit one register group (4 blocks = 1024 columns),
+//    so that all of them are requested before the programmatic-dependent-launch
+//    wait and none of their latency is exposed after it: ks >= K / 1024;
+//  * more than about two CTAs per SM per launch costs more than it gains: the
+//    launch then cannot be resident beside its neighbour in the stream, and its
+//    late CTAs start their weight loads only after the wait;
+//  * when the other stage of the forward has enough row tiles to fill the GPU on
+//    its own (1.5 per SM) and at most 8 tokens are in flight, this stage keeps
+//    to about one CTA per SM for the same reason, but splits K at least half as
+//    far as the first rule asks;
+//  * at least a quarter of the SMs should take part.
+// On a 4096 x 4096 layer at 1 bit/weight (k = 2048), batch 1, this split takes
+// 7.8 us per layer against 8.8 us for a plain "two CTAs per SM" split.
 struct DecodePlan {
   int rt, ks, piece;
   int64_t kchunk;
 };
 
-static DecodePlan plan_decode(int64_t M, int64_t K, int batch, int num_sms) {
-  // 64-row CTAs (4 warps, one 16-row tile each) and a K split that brings the
-  // CTA count to about two per SM.  A sweep of every (row tiles, K split)
-  // choice on B200 over the layer shapes of the workloads found this within
-  // about 5% of the best choice for each shape and batch.
+static DecodePlan plan_decode(int64_t M, int64_t K, int batch, int num_sms, int64_t peer_rows) {
   const int ntok = batch > 8 ? 16 : 8;
   const int nvalid = batch < ntok ? batch : ntok;
   const int64_t tiles = (M + 63) / 64;
-  int ks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kMaxClusterK, 2 * num_sms / tiles)));
+  const int64_t peer_tiles = (peer_rows + 63) / 64;
+  const int64_t ks_pref = std::min<int64_t>(kMaxClusterK, std::max<int64_t>(1, (K + 1023) / 1024));
+  const bool peer_fills = batch <= 8 && 2 * peer_tiles >= 3 * static_cast<int64_t>(num_sms);
+  const int64_t cap = peer_fills ? num_sms : 2 * num_sms;
+  int64_t ks = ks_pref;
+  while (ks > 1 && tiles * ks > cap) --ks;
+  if (peer_fills) ks = std::max(ks, (ks_pref + 1) / 2);  // long rows still need CTAs in flight
+  const int64_t ks_min = std::min<int64_t>(kMaxClusterK, (num_sms + 4 * tiles - 1) / (4 * tiles));
+  ks = std::max(ks, ks_min);
   int64_t kchunk = (K + ks - 1) / ks;
   kchunk = (kchunk + 255) / 256 * 256;
-  ks = static_cast<int>((K + kchunk - 1) / kchunk);
+  const int ks_eff = static_cast<int>((K + kchunk - 1) / kchunk);
   int piece = static_cast<int>(kchunk);
-  while (piece > 256 && dec_smem_layout(piece, nvalid, ntok, ks, 4).total > kSmemBudget) piece -= 256;
-  return DecodePlan{4, ks, piece, kchunk};
+  while (piece > 256 && dec_smem_layout(piece, nvalid, ntok, ks_eff, 4).total > kSmemBudget) piece -= 256;
+  return DecodePlan{4, ks_eff, piece, kchunk};
 }
 
 dbf_status launch_decode_stage(const DecodeArgs& args_in, bool class_expand, bool out_f32, const DeviceInfo& dev,
                                cudaStream_t stream) {
   DecodeArgs a = args_in;
-  const DecodePlan plan = plan_decode(a.M, a.K, a.batch, dev.num_sms);
+  const DecodePlan plan = plan_decode(a.M, a.K, a.batch, dev.num_sms, a.peer_rows);
   a.kchunk = static_cast<int>(plan.kchunk);
   if (a.batch > 8) return launch_rt<2, 4>(a, class_expand, out_f32, plan.ks, plan.piece, stream);
   return launch_rt<1, 4>(a, class_expand, out_f32, plan.ks, plan.piece, stream);
