@@ -31,6 +31,13 @@
 //   warps 10-13 epilogue: TMEM -> registers -> row scale -> a 32x32 transpose
 //               in shared memory -> 16-byte global stores (warp w reads TMEM
 //               lanes 32*(w%4) .. 32*(w%4)+31).
+// Few tiles (small batches): the K range of each 128 x 128 tile is split over a
+// cluster of 2-8 CTAs, one (tile, K slice) per CTA.  After the main loop each
+// CTA sorts its fp32 partial tile by destination rank into its idle A ring; a
+// cluster barrier says every ring is idle; one thread bulk-copies each peer its
+// slice into the peer's B ring (completion counted on the peer's mbarrier), and
+// every rank finishes its share of the token columns, adding the parts in rank
+// order.
 // Stage hand-off is through mbarriers; every wait is bounded and an expired
 // wait records DBF_ERR_TIMEOUT in the workspace status word, raises a CTA-wide
 // abort flag and lets all roles fall through to the teardown, which frees TMEM
@@ -39,7 +46,9 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <map>
 #include <mutex>
+#include <utility>
 #include <type_traits>
 
 #include "dbf_device.cuh"
@@ -58,22 +67,28 @@ constexpr int kWarpEpi0 = kWarpMma + 1;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kEpiStageBytes = 32 * 32 * 4;  // one warp's 32 tokens x 32 rows (fp32 worst case)
 
-template <int NTILE>
+template <int NTILE, bool SPLIT>
 struct Cfg {
   static constexpr int kStages = NTILE == 256 ? 4 : 6;
   static constexpr int kBBytes = NTILE * kBK * 2;
   static constexpr int kEpiOffset = kStages * (kABytes + kBBytes);
   static constexpr int kBarOffset = kEpiOffset + 4 * kEpiStageBytes;
-  // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done
-  static constexpr int kNumBars = 3 * kStages + 5;
+  // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done, recv
+  static constexpr int kNumBars = 3 * kStages + 6;
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;  // + tmem slot/abort + align slack
   static constexpr int kTmemCols = 2 * NTILE;
+  // split K: once a CTA's MMAs are done its operand ring is idle; the A ring
+  // then holds this CTA's fp32 partial tile sorted by destination rank and the
+  // B ring receives the peers' parts, both [rank][NTILE/ks/4][128 rows] float4.
+  static constexpr int kPartialBytes = kBM * NTILE * 4;
+  static_assert(!SPLIT || (kPartialBytes <= kStages * kABytes && kPartialBytes <= kStages * kBBytes),
+                "split-K partial tiles must fit in the idle operand ring");
 };
 
-template <int NTILE, bool KSCALE, bool OUT_F32>
+template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     dbf_prefill_gemm_kernel(const __grid_constant__ CUtensorMap act_map, const PrefillArgs p) {
-  using C = Cfg<NTILE>;
+  using C = Cfg<NTILE, SPLIT>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -87,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = bars + 3 * S;
   uint64_t* acc_empty = bars + 3 * S + 2;
   uint64_t* mma_done = bars + 3 * S + 4;
+  uint64_t* recv_bar = bars + 3 * S + 5;  // split K: the peers' parts have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -95,6 +111,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m_tiles = (p.M + kBM - 1) / kBM;
   const int num_tiles = m_tiles * ((p.batch + NTILE - 1) / NTILE);
   const int KT = p.K / kBK;
+  const int nblk = (KT + 3) / 4;
+  // Work items: (tile, K slice).  Without a split there is one slice per tile
+  // and the CTAs walk the items persistently; with a split, the ks CTAs of a
+  // cluster take the ks slices of one tile (one item per CTA) and add their
+  // partial sums through distributed shared memory.
+  const int ks = SPLIT ? static_cast<int>(cluster_size()) : 1;
+  const int rank = SPLIT ? static_cast<int>(cluster_rank()) : 0;
+  const int num_items = num_tiles * ks;
+  const int bper = (nblk + ks - 1) / ks;
+  auto item_blocks = [&](int w, int& b0, int& b1) {
+    b0 = min(nblk, (w % ks) * bper);
+    b1 = min(nblk, b0 + bper);
+  };
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
@@ -107,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[i], 128);
     }
     mbar_init(mma_done, 1);
+    mbar_init(recv_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -118,6 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Peers write into this CTA's receive buffer only after every CTA of the
+  // cluster has initialised its barriers (the matching wait comes later).
+  if constexpr (SPLIT) cluster_arrive_relaxed();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < kWarpTma) {
@@ -128,17 +161,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // holds words 4h..4h+3 (column pairs 4h..4h+3 of every group).
     const int r_local = tid & (kBM - 1);
     const int h = tid >> 7;
-    const int nblk = (KT + 3) / 4;
-    // block sequence of this CTA: (tile, blk) with blk fastest
-    int f_tile = blockIdx.x, f_blk = 0;
+    // block sequence of this CTA: (item, blk) with blk fastest
+    int f_w = blockIdx.x, f_blk = 0, f_end = 0;
+    auto f_seek = [&]() {
+      while (f_w < num_items) {
+        item_blocks(f_w, f_blk, f_end);
+        if (f_blk < f_end) return;
+        f_w += gridDim.x;
+      }
+    };
+    f_seek();
     auto fetch_next = [&]() -> uint4 {
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (f_tile < num_tiles) {
-        const int r = (f_tile % m_tiles) * kBM + r_local;
+      if (f_w < num_items) {
+        const int r = ((f_w / ks) % m_tiles) * kBM + r_local;
         if (r < p.M) v = ldg_stream_u4(p.packed + static_cast<int64_t>(r) * p.wpr + 8 * f_blk + 4 * h);
-        if (++f_blk == nblk) {
-          f_blk = 0;
-          f_tile += gridDim.x;
+        if (++f_blk == f_end) {
+          f_w += gridDim.x;
+          f_seek();
         }
       }
       return v;
@@ -148,24 +188,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 4; ++i)
         sc[i] = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 16 * i + 8 * h));
     };
+    int first_b0 = 0, first_b1 = 0;
+    if (static_cast<int>(blockIdx.x) < num_items) item_blocks(blockIdx.x, first_b0, first_b1);
+    const int kt_first = min(KT - 1, 4 * first_b0);
     uint4 w_n1, w_n2, wcur = make_uint4(0u, 0u, 0u, 0u);
     uint4 sc_next[4];
     if (p.weights_early) {
       w_n1 = fetch_next();
       w_n2 = fetch_next();
-      if constexpr (KSCALE) fetch_scale(0, sc_next);
+      if constexpr (KSCALE) fetch_scale(kt_first, sc_next);
     }
     pdl_wait();
     if (!p.weights_early) {
       w_n1 = fetch_next();
       w_n2 = fetch_next();
-      if constexpr (KSCALE) fetch_scale(0, sc_next);
+      if constexpr (KSCALE) fetch_scale(kt_first, sc_next);
     }
     bool ok = true;
     const int swz = r_local & 7;
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      for (int kt = 0; kt < KT; ++kt, ++it) {
+    for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
+      int b0, b1;
+      item_blocks(w, b0, b1);
+      const int kt0 = 4 * b0, kt1 = min(KT, 4 * b1);
+      for (int kt = kt0; kt < kt1; ++kt, ++it) {
         const int s = static_cast<int>(it % S);
         const uint32_t use = it / S;
         if ((kt & 3) == 0) {
@@ -177,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (KSCALE) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) sc[i] = sc_next[i];
-          fetch_scale(kt + 1 < KT ? kt + 1 : 0, sc_next);
+          // the next item of a persistent CTA starts again at K step 0
+          fetch_scale(kt + 1 < kt1 ? kt + 1 : (SPLIT ? kt0 : 0), sc_next);
         }
         if (it >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) {
           ok = false;
@@ -212,9 +259,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       pdl_wait();
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int n0 = (tile / m_tiles) * NTILE;
-        for (int kt = 0; kt < KT; ++kt, ++it) {
+      for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
+        int b0, b1;
+        item_blocks(w, b0, b1);
+        const int n0 = ((w / ks) / m_tiles) * NTILE;
+        for (int kt = 4 * b0; kt < min(KT, 4 * b1); ++kt, ++it) {
           const int s = static_cast<int>(it % S);
           const uint32_t use = it / S;
           if (it >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) {
@@ -233,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_f16_f32(kBM, NTILE);
       bool ok = true;
       uint32_t it = 0, local = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x, ++local) {
         const uint32_t buf = local & 1;
         if (local >= 2 && !mbar_wait_bounded(&acc_empty[buf], ((local >> 1) - 1) & 1, abort_flag, p.status)) {
           ok = false;
@@ -241,7 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * NTILE;
-        for (int kt = 0; kt < KT; ++kt, ++it) {
+        int b0, b1;
+        item_blocks(w, b0, b1);
+        const int kt0 = 4 * b0, kt1 = min(KT, 4 * b1);
+        for (int kt = kt0; kt < kt1; ++kt, ++it) {
           const int s = static_cast<int>(it % S);
           const uint32_t par = (it / S) & 1;
           if (!mbar_wait_bounded(&full_a[s], par, abort_flag, p.status) ||
@@ -255,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             tc_mma_f16_ss(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32), smem_desc_sw128_kmajor(b_addr + kk * 32),
-                          idesc, (kt | kk) != 0 ? 1u : 0u);
+                          idesc, (kt != kt0 || kk != 0) ? 1u : 0u);
           }
           tc_commit(&empty[s]);
         }
@@ -266,71 +318,162 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------ epilogue
     using OutT = typename std::conditional<OUT_F32, float, __half>::type;
-    constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
-    const int q = warp & 3;                  // TMEM lane quadrant this warp may access
-    OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
     OutT* out = static_cast<OutT*>(p.out);
-    const bool ld_ok = (p.ld_out % kVec) == 0;
     uint32_t local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const uint32_t buf = local & 1;
-      if (!mbar_wait_bounded(&acc_full[buf], (local >> 1) & 1, abort_flag, p.status)) break;
+    if constexpr (SPLIT) {
+      // Reduce-scatter of the ks partial tiles of one (tile, all K) item: rank j
+      // finishes token columns [j*cw, (j+1)*cw).  Each thread (one weight row)
+      // sorts its partial row into the idle A ring by destination rank; after a
+      // cluster barrier (every rank's MMAs are done, so every ring is free) one
+      // thread sends each peer its slice with a bulk copy that completes on the
+      // peer's mbarrier, and each rank adds the ks parts of its own columns in
+      // rank order (deterministic).
+      const int cw = NTILE / ks;
+      const int cw4 = cw / 4;
+      const uint32_t slice_bytes = static_cast<uint32_t>(kBM * cw * 4);
+      float4* part = reinterpret_cast<float4*>(a_st);  // [dst rank][cw4][128 rows]
+      float4* recv = reinterpret_cast<float4*>(b_st);  // [src rank][cw4][128 rows]
+      const int r = q * 32 + lane;
+      const int w = blockIdx.x;  // one item per CTA
+      const bool got = mbar_wait_bounded(&acc_full[0], 0, abort_flag, p.status);
       tc_fence_after();
-      const int m0 = (tile % m_tiles) * kBM;
-      const int n0 = (tile / m_tiles) * NTILE;
-      const int row0 = m0 + q * 32;
-      const int row = row0 + lane;
-      const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;
-      const bool rows_full = row0 + 32 <= p.M;
+      int b0, b1;
+      item_blocks(w, b0, b1);
+      const bool have = got && b1 > b0;  // an empty K slice contributes zeros
       for (int col = 0; col < NTILE; col += 32) {
-        if (n0 + col >= p.batch) break;  // warp-uniform
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * NTILE + static_cast<uint32_t>(col),
-                           v);
-        tmem_ld_wait();
-        const int tok0 = n0 + col;
-        if (rows_full && ld_ok && tok0 + 32 <= p.batch) {
-          // transpose through shared memory, then 16-byte stores of kVec consecutive rows
+        if (have) {
+          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col), v);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float val = rs * __uint_as_float(v[j]);
-            if constexpr (OUT_F32) {
-              stg[j * 32 + lane] = val;
-            } else {
-              stg[j * 32 + lane] = __float2half_rn(val);
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const int c = col + 4 * j4;
+          const int dst = c / cw, cc = c - dst * cw;
+          part[(dst * cw4 + (cc >> 2)) * kBM + r] =
+              make_float4(__uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]), __uint_as_float(v[4 * j4 + 2]),
+                          __uint_as_float(v[4 * j4 + 3]));
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();  // the partial tile is read by the bulk copies
+      cluster_wait_acquire();    // phase 0: every CTA of the cluster initialised its barriers
+      cluster_arrive_release();  // phase 1: this CTA's MMAs are done and its partial tile is written
+      cluster_wait_acquire();
+      if (tid == kWarpEpi0 * 32) {
+        mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(ks - 1) * slice_bytes);
+        for (int j = 1; j < ks; ++j) {
+          const int dst = (rank + j) % ks;
+          bulk_copy_to_peer(map_to_rank(recv + rank * cw4 * kBM, static_cast<uint32_t>(dst)), part + dst * cw4 * kBM,
+                            slice_bytes, map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
+        }
+      }
+      if (mbar_wait_cluster_bounded(recv_bar, 0, p.status)) {
+        const int m0 = ((w / ks) % m_tiles) * kBM;
+        const int n0 = ((w / ks) / m_tiles) * NTILE + rank * cw;
+        const int row = m0 + r;
+        if (row < p.M) {
+          const float rs = __half2float(p.rowscale[row]);
+          for (int c4 = 0; c4 < cw4; ++c4) {
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int src = 0; src < ks; ++src) {
+              const float4 t = src == rank ? part[(rank * cw4 + c4) * kBM + r] : recv[(src * cw4 + c4) * kBM + r];
+              sum.x += t.x;
+              sum.y += t.y;
+              sum.z += t.z;
+              sum.w += t.w;
             }
-          }
-          __syncwarp();
-          constexpr int kChunksPerTok = 32 / kVec;
+            const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
-          for (int m = 0; m < 32 * kChunksPerTok / 32; ++m) {
-            const int cidx = lane + 32 * m;
-            const int tk = cidx / kChunksPerTok, rp = cidx % kChunksPerTok;
-            const uint4 val = *reinterpret_cast<const uint4*>(stg + tk * 32 + rp * kVec);
-            *reinterpret_cast<uint4*>(out + static_cast<int64_t>(tok0 + tk) * p.ld_out + row0 + rp * kVec) = val;
-          }
-          __syncwarp();
-        } else if (row < p.M) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tok = tok0 + j;
-            if (tok < p.batch) {
-              const float val = rs * __uint_as_float(v[j]);
-              if constexpr (OUT_F32) {
-                out[static_cast<int64_t>(tok) * p.ld_out + row] = val;
-              } else {
-                out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(val);
+            for (int e = 0; e < 4; ++e) {
+              const int tok = n0 + 4 * c4 + e;
+              if (tok < p.batch) {
+                if constexpr (OUT_F32) {
+                  out[static_cast<int64_t>(tok) * p.ld_out + row] = rs * vals[e];
+                } else {
+                  out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(rs * vals[e]);
+                }
               }
             }
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
+    } else {
+      constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
+      OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
+      const bool ld_ok = (p.ld_out % kVec) == 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+        const uint32_t buf = local & 1;
+        if (!mbar_wait_bounded(&acc_full[buf], (local >> 1) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const int m0 = (tile % m_tiles) * kBM;
+        const int n0 = (tile / m_tiles) * NTILE;
+        const int row0 = m0 + q * 32;
+        const int row = row0 + lane;
+        const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;
+        const bool rows_full = row0 + 32 <= p.M;
+        for (int col = 0; col < NTILE; col += 32) {
+          if (n0 + col >= p.batch) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * NTILE + static_cast<uint32_t>(col),
+                             v);
+          tmem_ld_wait();
+          const int tok0 = n0 + col;
+          if (rows_full && ld_ok && tok0 + 32 <= p.batch) {
+            // transpose through shared memory, then 16-byte stores of kVec consecutive rows
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float val = rs * __uint_as_float(v[j]);
+              if constexpr (OUT_F32) {
+                stg[j * 32 + lane] = val;
+              } else {
+                stg[j * 32 + lane] = __float2half_rn(val);
+              }
+            }
+            __syncwarp();
+            constexpr int kChunksPerTok = 32 / kVec;
+#pragma unroll
+            for (int m = 0; m < 32 * kChunksPerTok / 32; ++m) {
+              const int cidx = lane + 32 * m;
+              const int tk = cidx / kChunksPerTok, rp = cidx % kChunksPerTok;
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + tk * 32 + rp * kVec);
+              *reinterpret_cast<uint4*>(out + static_cast<int64_t>(tok0 + tk) * p.ld_out + row0 + rp * kVec) = val;
+            }
+            __syncwarp();
+          } else if (row < p.M) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = tok0 + j;
+              if (tok < p.batch) {
+                const float val = rs * __uint_as_float(v[j]);
+                if constexpr (OUT_F32) {
+                  out[static_cast<int64_t>(tok) * p.ld_out + row] = val;
+                } else {
+                  out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(val);
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+      }
     }
   }
 
   // ------------------------------------------------ teardown
+  if constexpr (SPLIT) {
+    if (warp < kWarpEpi0) {  // the epilogue warps passed phases 0 and 1 above
+      __syncwarp();
+      cluster_wait_acquire();
+      cluster_arrive_release();
+      cluster_wait_acquire();
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
@@ -340,6 +483,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     (void)mbar_wait_bounded(mma_done, 0, abort_flag, p.status);
     __syncwarp();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if constexpr (SPLIT) {
+    // phase 2: no CTA leaves while a peer's bulk copy may still read from or
+    // write into its shared memory (every rank has waited for its own parts)
+    cluster_arrive_release();
+    cluster_wait_acquire();
   }
 }
 
@@ -358,36 +507,101 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int NTILE, bool KSCALE, bool OUT_F32>
-dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, const DeviceInfo& dev, cudaStream_t stream) {
-  auto kernel = dbf_prefill_gemm_kernel<NTILE, KSCALE, OUT_F32>;
-  constexpr int smem = Cfg<NTILE>::kSmemBytes;
+template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32>
+dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, const DeviceInfo& dev,
+                        cudaStream_t stream) {
+  auto kernel = dbf_prefill_gemm_kernel<NTILE, SPLIT, KSCALE, OUT_F32>;
+  constexpr int smem = Cfg<NTILE, SPLIT>::kSmemBytes;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return DBF_ERR_CUDA;
   const int64_t m_tiles = (a.M + kBM - 1) / kBM;
   const int64_t n_tiles = (a.batch + NTILE - 1) / NTILE;
-  const int64_t grid = std::min<int64_t>(m_tiles * n_tiles, dev.num_sms);
+  // split K: one (tile, K slice) item per CTA, the ks slices of a tile in one cluster
+  const int64_t grid = SPLIT ? m_tiles * n_tiles * ks : std::min<int64_t>(m_tiles * n_tiles, dev.num_sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(SPLIT ? ks : 1);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, map, a) == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
+template <int NTILE, bool SPLIT>
+dbf_status launch_split(const PrefillArgs& a, const CUtensorMap& map, int ks, bool out_f32, const DeviceInfo& dev,
+                        cudaStream_t stream) {
+  if (a.kscale != nullptr)
+    return out_f32 ? launch_typed<NTILE, SPLIT, true, true>(a, map, ks, dev, stream)
+                   : launch_typed<NTILE, SPLIT, true, false>(a, map, ks, dev, stream);
+  return out_f32 ? launch_typed<NTILE, SPLIT, false, true>(a, map, ks, dev, stream)
+                 : launch_typed<NTILE, SPLIT, false, false>(a, map, ks, dev, stream);
+}
+
 }  // namespace
+
+// Tile shape and K split.  128 x 128 tiles with no split when there are enough
+// of them to occupy half the SMs (128 x 256 past 128 tokens); otherwise the K
+// range of each 128 x 128 tile is split over a cluster of 2, 4 or 8 CTAs: as
+// many as fit on the SMs, at most one slice per 256-column block, and no more
+// clusters than the GPU can hold at once (a second wave would double the time).
+static int prefill_k_split(int64_t M, int64_t K, int64_t batch, int num_sms) {
+  const int64_t tiles128 = (M + kBM - 1) / kBM * ((batch + 127) / 128);
+  const int64_t nblk = (K / kBK + 3) / 4;
+  if (2 * tiles128 > num_sms) return 1;
+  int ks = 1;
+  while (ks < 8 && tiles128 * ks * 2 <= num_sms && ks * 2 <= nblk) ks *= 2;
+  return ks;
+}
+
+// Clusters of ks split-K CTAs that can be resident at once (0 if unknown).
+static int max_resident_clusters(int device, int ks, int num_sms) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(device, ks);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  auto kernel = dbf_prefill_gemm_kernel<128, true, false, false>;
+  constexpr int smem = Cfg<128, true>::kSmemBytes;
+  int n = 0;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ks * num_sms), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+  }
+  cache[key] = n;
+  return n;
+}
 
 dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t act_rows, bool out_f32,
                                const DeviceInfo& dev, cudaStream_t stream) {
   auto encode = encode_fn();
   if (!encode) return DBF_ERR_CUDA;
-  const int ntile = a.batch > 128 ? 256 : 128;
-  if (static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + ntile - 1) / ntile) > 0x7fffffffLL)
+  int ks = prefill_k_split(a.M, a.K, a.batch, dev.num_sms);
+  const int64_t tiles128 = static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + 127) / 128);
+  while (ks > 1 && tiles128 > max_resident_clusters(dev.device, ks, dev.num_sms)) ks /= 2;
+  const int ntile = (ks == 1 && a.batch > 128) ? 256 : 128;
+  if (static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + ntile - 1) / ntile) * ks > 0x7fffffffLL)
     return DBF_ERR_UNSUPPORTED_SHAPE;
 
   CUtensorMap map;
@@ -400,13 +614,9 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return DBF_ERR_CUDA;
 
-  const bool ks = a.kscale != nullptr;
-  if (ntile == 256) {
-    if (ks) return out_f32 ? launch_typed<256, true, true>(a, map, dev, stream) : launch_typed<256, true, false>(a, map, dev, stream);
-    return out_f32 ? launch_typed<256, false, true>(a, map, dev, stream) : launch_typed<256, false, false>(a, map, dev, stream);
-  }
-  if (ks) return out_f32 ? launch_typed<128, true, true>(a, map, dev, stream) : launch_typed<128, true, false>(a, map, dev, stream);
-  return out_f32 ? launch_typed<128, false, true>(a, map, dev, stream) : launch_typed<128, false, false>(a, map, dev, stream);
+  if (ks > 1) return launch_split<128, true>(a, map, ks, out_f32, dev, stream);
+  if (ntile == 256) return launch_split<256, false>(a, map, 1, out_f32, dev, stream);
+  return launch_split<128, false>(a, map, 1, out_f32, dev, stream);
 }
 
 }  // namespace dbf
