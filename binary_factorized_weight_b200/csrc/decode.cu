@@ -291,30 +291,54 @@ __global__ void __launch_bounds__(kDecThreads, 1) dbf_decode_stage_kernel(const 
     // ---- sign products over this warp's slice of the piece
     for (int gb = sb0; gb < sb1; gb += D) {
       if (gb + D < sb1) load_group(wb, gb + D, sb1);
+      if (gb + D <= sb1 && pe - (gb + D) * 256 >= 0) {
+        // D whole blocks: fixed offsets and no per-step predicates
+        const int off0 = (gb * 256 - pk) >> 1;
 #pragma unroll
-      for (int d = 0; d < D; ++d) {
-        const int blk = gb + d;
-        if (blk < sb1) {
-          const int off = (blk * 256 - pk) >> 1;  // word offset of the block in a staged row
-          const int nsteps = min(16, (pe - blk * 256) >> 4);
-          // all of the block's activation fragments first, so the shared-memory
-          // loads overlap each other instead of each MMA waiting for its own
+        for (int d = 0; d < D; ++d) {
           uint2 bb[16][NT];
 #pragma unroll
           for (int s = 0; s < 16; ++s)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              bb[s][nt] = s < nsteps ? *reinterpret_cast<const uint2*>(arow[nt] + off + 8 * s) : make_uint2(0u, 0u);
+              bb[s][nt] = *reinterpret_cast<const uint2*>(arow[nt] + off0 + 128 * d + 8 * s);
 #pragma unroll
           for (int s = 0; s < 16; ++s) {
-            if (s < nsteps) {
-              const uint32_t a0 = form_pair<CLASS>(wa[d][0].x, s);
-              const uint32_t a2 = form_pair<CLASS>(wa[d][0].y, s);
-              const uint32_t a1 = form_pair<CLASS>(wa[d][1].x, s);
-              const uint32_t a3 = form_pair<CLASS>(wa[d][1].y, s);
+            const uint32_t a0 = form_pair<CLASS>(wa[d][0].x, s);
+            const uint32_t a2 = form_pair<CLASS>(wa[d][0].y, s);
+            const uint32_t a1 = form_pair<CLASS>(wa[d][1].x, s);
+            const uint32_t a3 = form_pair<CLASS>(wa[d][1].y, s);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              mma_m16n8k16(acc[CLASS ? s : (s & 3)][nt], a0, a1, a2, a3, bb[s][nt].x, bb[s][nt].y);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          const int blk = gb + d;
+          if (blk < sb1) {
+            const int off = (blk * 256 - pk) >> 1;  // word offset of the block in a staged row
+            const int nsteps = min(16, (pe - blk * 256) >> 4);
+            // all of the block's activation fragments first, so the shared-memory
+            // loads overlap each other instead of each MMA waiting for its own
+            uint2 bb[16][NT];
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
-                mma_m16n8k16(acc[CLASS ? s : (s & 3)][nt], a0, a1, a2, a3, bb[s][nt].x, bb[s][nt].y);
+                bb[s][nt] = s < nsteps ? *reinterpret_cast<const uint2*>(arow[nt] + off + 8 * s) : make_uint2(0u, 0u);
+#pragma unroll
+            for (int s = 0; s < 16; ++s) {
+              if (s < nsteps) {
+                const uint32_t a0 = form_pair<CLASS>(wa[d][0].x, s);
+                const uint32_t a2 = form_pair<CLASS>(wa[d][0].y, s);
+                const uint32_t a1 = form_pair<CLASS>(wa[d][1].x, s);
+                const uint32_t a3 = form_pair<CLASS>(wa[d][1].y, s);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                  mma_m16n8k16(acc[CLASS ? s : (s & 3)][nt], a0, a1, a2, a3, bb[s][nt].x, bb[s][nt].y);
+              }
             }
           }
         }
