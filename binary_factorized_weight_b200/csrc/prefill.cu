@@ -600,7 +600,14 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
   int ks = prefill_k_split(a.M, a.K, a.batch, dev.num_sms);
   const int64_t tiles128 = static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + 127) / 128);
   while (ks > 1 && tiles128 > max_resident_clusters(dev.device, ks, dev.num_sms)) ks /= 2;
-  const int ntile = (ks == 1 && a.batch > 128) ? 256 : 128;
+  // Past 128 tokens, 256-token tiles, unless they would keep fewer than half
+  // the SMs busy (few weight rows): then 128-token tiles, which double the
+  // tiles at the price of expanding each weight tile twice as often.
+  int ntile = 128;
+  if (ks == 1 && a.batch > 128) {
+    const int64_t tiles256 = static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + 255) / 256);
+    ntile = 2 * tiles256 <= dev.num_sms ? 128 : 256;
+  }
   if (static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + ntile - 1) / ntile) * ks > 0x7fffffffLL)
     return DBF_ERR_UNSUPPORTED_SHAPE;
 
