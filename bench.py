@@ -274,6 +274,41 @@ class Workload:
         return g
 
 
+GROUPS = {"qkv": ("q", "k", "v"), "gate_up": ("gate", "up")}
+
+
+class GroupWorkload(Workload):
+    """R rotated copies of layers that share their input, run through dbf_forward_grouped."""
+
+    def __init__(self, dbf, torch, shapes, batch, device, copies=None):
+        self.dbf, self.torch = dbf, torch
+        self.batch = batch
+        self.m_in = shapes[0].m_in
+        d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        Ls = [gen.make_layer(s, batch) for s in shapes]
+        self.host = Ls
+        base = [dict(packedA=dbf.dbf_pack_signs(d(L["A"])), packedB=dbf.dbf_pack_signs(d(L["B"])), a=d(L["a"]),
+                     m=d(L["mid"]), b=d(L["b"]), n=s.n, k=s.k) for s, L in zip(shapes, Ls)]
+        self.bytes = sum(layer_bytes(s.n, s.k, s.m_in, batch) for s in shapes) - 2 * batch * self.m_in * (
+            len(shapes) - 1)  # x is read once
+        self.flops = sum(layer_flops(s.n, s.k, s.m_in, batch) for s in shapes)
+        weight_bytes = sum((L["packedA"].numel() + L["packedB"].numel()) * 4 + 2 * (L["n"] + L["k"] + self.m_in)
+                           for L in base)
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        self.copies = copies or max(2, int(math.ceil(4 * l2 / weight_bytes)))
+        self.groups = [base] + [[{k: (v.clone() if hasattr(v, "clone") else v) for k, v in L.items()} for L in base]
+                                for _ in range(self.copies - 1)]
+        self.x = d(Ls[0]["x"])
+        self.ys = [torch.empty((batch, s.n), dtype=torch.float16, device=device) for s in shapes]
+        self.ws = dbf.dbf_new_grouped_workspace(base, self.m_in, batch, device=device)
+        self.flags = dbf.DBF_FWD_WEIGHTS_STATIC
+        self.path = "decode (grouped)" if batch <= 16 else "prefill (per layer)"
+
+    def forward_all(self, x=None, y=None):
+        for grp in self.groups:
+            self.dbf.dbf_forward_grouped(self.x, grp, self.m_in, ys=self.ys, workspace=self.ws, flags=self.flags)
+
+
 def run_ours(args, shape, batch):
     import torch
 
@@ -522,6 +557,41 @@ def run_sweep(args):
         print(json.dumps(row), flush=True)
         del g, wl
         torch.cuda.empty_cache()
+    # layers that share their input, as one grouped forward, against the same
+    # layers run one by one (the rows above)
+    by_name = {(r["layer"], r["batch"]): r["us"] for r in rows}
+    for bits in (1, 2):
+        set_ = {s.name.split("_")[0]: s for s in gen.LAYER_SET[bits]}
+        for gname, members in GROUPS.items():
+            shapes = [set_[m] for m in members]
+            for batch in (1, 16):
+                wl = GroupWorkload(dbf, torch, shapes, batch, device)
+                g = wl.capture()
+                for _ in range(5):
+                    g.replay()
+                torch.cuda.synchronize()
+                reps = max(3, int(200 / max(1, wl.copies)))
+                times = []
+                for _ in range(7):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    times.append(e0.elapsed_time(e1) / reps / wl.copies * 1e3)
+                us = statistics.median(times)
+                sep = sum(by_name.get((s.name, batch), float("nan")) for s in shapes)
+                gbs = wl.bytes / (us * 1e-6) / 1e9
+                row = {"layer": f"{gname}_{bits}b (grouped)", "members": [s.name for s in shapes], "batch": batch,
+                       "us": us, "us_p10": sorted(times)[0], "us_p90": sorted(times)[-1],
+                       "tokens_per_s": batch / (us * 1e-6), "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                       "tflops": wl.flops / (us * 1e-6) / 1e12, "copies": wl.copies, "path": wl.path,
+                       "separate_layers_us": sep, "speedup_vs_separate": sep / us}
+                rows.append(row)
+                print(json.dumps(row), flush=True)
+                del g, wl
+                torch.cuda.empty_cache()
     with open(args.sweep, "w") as f:
         json.dump({"peaks": peaks, "rows": rows}, f, indent=1)
 

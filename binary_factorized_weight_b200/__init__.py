@@ -30,6 +30,7 @@ __all__ = [
     "dbf_packed_words_per_row", "dbf_packed_words", "dbf_pack_signs",
     "dbf_forward_workspace_bytes", "dbf_new_workspace", "dbf_forward",
     "dbf_reconstruct_dense", "dbf_workspace_status", "dbf_status_string", "dbf_forward_noalloc",
+    "DBF_MAX_GROUP", "dbf_forward_grouped_workspace_bytes", "dbf_new_grouped_workspace", "dbf_forward_grouped",
 ]
 
 DBF_I8, DBF_F16, DBF_F32 = 0, 1, 2
@@ -52,8 +53,21 @@ EXPORTED_SYMBOLS = (
     "dbf_reconstruct_dense",
     "dbf_workspace_status",
     "dbf_forward_noalloc",
+    "dbf_forward_grouped_workspace_bytes",
+    "dbf_forward_grouped",
     "dbf_status_string",
 )
+
+DBF_MAX_GROUP = 8
+
+
+class _LayerDesc(ctypes.Structure):
+    """struct dbf_layer_desc of include/dbf.h."""
+    _fields_ = [
+        ("packedA", ctypes.c_void_p), ("packedB", ctypes.c_void_p),
+        ("a", ctypes.c_void_p), ("m", ctypes.c_void_p), ("b", ctypes.c_void_p),
+        ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("y", ctypes.c_void_p),
+    ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -95,6 +109,10 @@ def load_library():
     lib.dbf_workspace_status.restype = i32
     lib.dbf_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, u32, vp]
     lib.dbf_forward_noalloc.restype = i32
+    lib.dbf_forward_grouped_workspace_bytes.argtypes = [ctypes.POINTER(_LayerDesc), i32, i64, i64]
+    lib.dbf_forward_grouped_workspace_bytes.restype = sz
+    lib.dbf_forward_grouped.argtypes = [vp, i64, i64, ctypes.POINTER(_LayerDesc), i32, i32, vp, sz, u32, vp]
+    lib.dbf_forward_grouped.restype = i32
     lib.dbf_status_string.argtypes = [i32]
     lib.dbf_status_string.restype = ctypes.c_char_p
     _LIB = lib
@@ -225,3 +243,44 @@ def dbf_workspace_status(workspace: torch.Tensor, stream=None) -> int:
     _check("dbf_workspace_status", load_library().dbf_workspace_status(
         _ptr(workspace), _stream(stream), ctypes.byref(out)))
     return int(out.value)
+
+
+def _layer_array(layers, ys=None):
+    arr = (_LayerDesc * len(layers))()
+    for i, L in enumerate(layers):
+        y = None if ys is None else ys[i]
+        arr[i] = _LayerDesc(L["packedA"].data_ptr(), L["packedB"].data_ptr(), L["a"].data_ptr(), L["m"].data_ptr(),
+                            L["b"].data_ptr(), int(L["n"]), int(L["k"]), None if y is None else y.data_ptr())
+    return arr
+
+
+def dbf_forward_grouped_workspace_bytes(layers, m_in: int, batch: int) -> int:
+    """Workspace bytes for dbf_forward_grouped over `layers` (dicts with at least n and k)."""
+    arr = (_LayerDesc * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i].n, arr[i].k = int(L["n"]), int(L["k"])
+    return int(load_library().dbf_forward_grouped_workspace_bytes(arr, len(layers), int(m_in), int(batch)))
+
+
+def dbf_new_grouped_workspace(layers, m_in: int, batch: int, device="cuda") -> torch.Tensor:
+    return torch.zeros(dbf_forward_grouped_workspace_bytes(layers, m_in, batch), dtype=torch.uint8, device=device)
+
+
+def dbf_forward_grouped(x: torch.Tensor, layers, m_in: int, ys=None, y_dtype: torch.dtype = torch.float16,
+                        workspace: Optional[torch.Tensor] = None, flags: int = 0, stream=None):
+    """Layers that share the input x: layers is a list of dicts with packedA, packedB, a, m, b (CUDA tensors)
+    and n, k; returns the list of outputs (batch x n_g each)."""
+    if x.dtype != torch.float16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp16 batch x m_in tensor")
+    batch = x.shape[0]
+    if x.shape[1] != m_in:
+        raise ValueError("x.shape[1] != m_in")
+    if ys is None:
+        ys = [torch.empty((batch, int(L["n"])), dtype=y_dtype, device=x.device) for L in layers]
+    if workspace is None:
+        workspace = dbf_new_grouped_workspace(layers, m_in, batch, device=x.device)
+    arr = _layer_array(layers, ys)
+    _check("dbf_forward_grouped", load_library().dbf_forward_grouped(
+        _ptr(x), int(m_in), int(batch), arr, len(layers), _dtype_code(ys[0].dtype), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), int(flags), _stream(stream)))
+    return ys

@@ -206,6 +206,143 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
   return launch_prefill_gemm(g2, V, batch, out_f32, dev, stream);
 }
 
+static size_t grouped_v_offset(const dbf_layer_desc* layers, int g, int64_t batch) {
+  size_t off = kStatusBytes;
+  for (int h = 0; h < g; ++h) off += (static_cast<size_t>(batch) * static_cast<size_t>(layers[h].k) * 2 + 255) / 256 * 256;
+  return off;
+}
+
+size_t dbf_forward_grouped_workspace_bytes(const dbf_layer_desc* layers, int num_layers, int64_t m_in,
+                                           int64_t batch) {
+  if (!layers || num_layers < 1 || num_layers > DBF_MAX_GROUP || m_in < 1 || batch < 1) return 0;
+  for (int g = 0; g < num_layers; ++g)
+    if (layers[g].n < 1 || layers[g].k < 1) return 0;
+  return grouped_v_offset(layers, num_layers, batch);
+}
+
+dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, const dbf_layer_desc* layers,
+                               int num_layers, dbf_dtype y_t, void* workspace, size_t ws_bytes, uint32_t flags,
+                               struct CUstream_st* stream_handle) {
+  if (!x || !layers) return DBF_ERR_INVALID_ARG;
+  if (num_layers < 1 || num_layers > DBF_MAX_GROUP) return DBF_ERR_INVALID_ARG;
+  for (int g = 0; g < num_layers; ++g) {
+    const dbf_layer_desc& l = layers[g];
+    if (!l.y) return DBF_ERR_INVALID_ARG;
+    dbf_status st = validate_factors(l.packedA, l.packedB, l.a, l.m, l.b, l.n, l.k, m_in);
+    if (st != DBF_OK) return st;
+    if (!aligned16(l.y)) return DBF_ERR_MISALIGNED;
+  }
+  if (batch < 1) return DBF_ERR_INVALID_ARG;
+  if (batch > kMaxRows) return DBF_ERR_UNSUPPORTED_SHAPE;
+  if (y_t != DBF_F16 && y_t != DBF_F32) return DBF_ERR_INVALID_ARG;
+  const uint32_t known = DBF_FWD_WEIGHTS_STATIC | DBF_FWD_FORCE_DECODE | DBF_FWD_FORCE_PREFILL |
+                         DBF_FWD_DECODE_SHIFT_EXPAND;
+  if ((flags & ~known) != 0) return DBF_ERR_INVALID_ARG;
+  if ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)) return DBF_ERR_INVALID_ARG;
+  if (!aligned16(x)) return DBF_ERR_MISALIGNED;
+  if (!workspace || !aligned16(workspace) ||
+      ws_bytes < dbf_forward_grouped_workspace_bytes(layers, num_layers, m_in, batch))
+    return DBF_ERR_WORKSPACE;
+  DeviceInfo dev;
+  dbf_status st = current_device(&dev);
+  if (st != DBF_OK) return st;
+
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_handle);
+  const bool out_f32 = y_t == DBF_F32;
+  const bool early = (flags & DBF_FWD_WEIGHTS_STATIC) != 0;
+  int* status = static_cast<int*>(workspace);
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  const size_t y_elt = out_f32 ? 4 : 2;
+  __half* V[DBF_MAX_GROUP];
+  int64_t rows_a = 0, rows_b = 0;
+  for (int g = 0; g < num_layers; ++g) {
+    V[g] = reinterpret_cast<__half*>(static_cast<char*>(workspace) + grouped_v_offset(layers, g, batch));
+    rows_a += layers[g].n;
+    rows_b += layers[g].k;
+  }
+
+  const bool decode = (flags & DBF_FWD_FORCE_DECODE) || (!(flags & DBF_FWD_FORCE_PREFILL) && batch <= 16);
+  if (decode) {
+    const bool class_expand = (flags & DBF_FWD_DECODE_SHIFT_EXPAND) == 0;
+    for (int64_t t0 = 0; t0 < batch; t0 += 16) {
+      const int nb = static_cast<int>(batch - t0 < 16 ? batch - t0 : 16);
+      DecodeGroup gb{};
+      DecodeGroup ga{};
+      gb.n = ga.n = num_layers;
+      for (int g = 0; g < num_layers; ++g) {
+        const dbf_layer_desc& l = layers[g];
+        DecodeArgs& sb = gb.layer[g];
+        sb.packed = l.packedB;
+        sb.wpr = words_per_row(m_in);
+        sb.M = static_cast<int>(l.k);
+        sb.K = static_cast<int>(m_in);
+        sb.act = xh + t0 * m_in;
+        sb.ld_act = m_in;
+        sb.kscale = reinterpret_cast<const __half*>(l.b);
+        sb.rowscale = reinterpret_cast<const __half*>(l.m);
+        sb.out = V[g] + t0 * l.k;
+        sb.ld_out = l.k;
+        sb.batch = nb;
+        sb.weights_early = early ? 1 : 0;
+        sb.status = status;
+        DecodeArgs& sa = ga.layer[g];
+        sa.packed = l.packedA;
+        sa.wpr = words_per_row(l.k);
+        sa.M = static_cast<int>(l.n);
+        sa.K = static_cast<int>(l.k);
+        sa.act = V[g] + t0 * l.k;
+        sa.ld_act = l.k;
+        sa.kscale = nullptr;
+        sa.rowscale = reinterpret_cast<const __half*>(l.a);
+        sa.out = static_cast<char*>(l.y) + static_cast<size_t>(t0) * static_cast<size_t>(l.n) * y_elt;
+        sa.ld_out = l.n;
+        sa.batch = nb;
+        sa.weights_early = 1;  // the stage-B launch releases this one only after its own wait
+        sa.status = status;
+      }
+      st = launch_decode_group(gb, rows_a, class_expand, /*out_f32=*/false, dev, stream);
+      if (st != DBF_OK) return st;
+      st = launch_decode_group(ga, rows_b, class_expand, out_f32, dev, stream);
+      if (st != DBF_OK) return st;
+    }
+    return DBF_OK;
+  }
+
+  // Large batches are tensor-core bound: one layer after the other.
+  for (int g = 0; g < num_layers; ++g) {
+    const dbf_layer_desc& l = layers[g];
+    PrefillArgs g1{};
+    g1.packed = l.packedB;
+    g1.wpr = words_per_row(m_in);
+    g1.M = static_cast<int>(l.k);
+    g1.K = static_cast<int>(m_in);
+    g1.kscale = reinterpret_cast<const __half*>(l.b);
+    g1.rowscale = reinterpret_cast<const __half*>(l.m);
+    g1.out = V[g];
+    g1.ld_out = l.k;
+    g1.batch = static_cast<int>(batch);
+    g1.weights_early = early ? 1 : 0;
+    g1.status = status;
+    st = launch_prefill_gemm(g1, xh, batch, /*out_f32=*/false, dev, stream);
+    if (st != DBF_OK) return st;
+    PrefillArgs g2{};
+    g2.packed = l.packedA;
+    g2.wpr = words_per_row(l.k);
+    g2.M = static_cast<int>(l.n);
+    g2.K = static_cast<int>(l.k);
+    g2.kscale = nullptr;
+    g2.rowscale = reinterpret_cast<const __half*>(l.a);
+    g2.out = l.y;
+    g2.ld_out = l.n;
+    g2.batch = static_cast<int>(batch);
+    g2.weights_early = 1;
+    g2.status = status;
+    st = launch_prefill_gemm(g2, V[g], batch, out_f32, dev, stream);
+    if (st != DBF_OK) return st;
+  }
+  return DBF_OK;
+}
+
 dbf_status dbf_reconstruct_dense(const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
                                  const uint16_t* m, const uint16_t* b, int64_t n, int64_t k, int64_t m_in, void* W,
                                  dbf_dtype W_t, struct CUstream_st* stream) {

@@ -56,6 +56,23 @@ dbf_status current_device(DeviceInfo* info);
 dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
                                cudaStream_t stream);
 
+// Several decode stages in one launch (layers that share their input: the
+// stage-B products of q, k and v, say, or their stage-A products).  Each layer's
+// rows are padded to whole 64-row CTA tiles; tile t belongs to the layer g with
+// tile_start[g] <= t < tile_start[g+1].  All layers share the kernel variant
+// (batch, kscale or not, output type) and the K split of the launch.
+constexpr int kMaxGroup = 8;
+struct DecodeGroup {
+  int n;
+  int tile_start[kMaxGroup + 1];
+  DecodeArgs layer[kMaxGroup];
+};
+
+// Fills tile_start and each layer's kchunk, then launches.  peer_rows: rows of
+// the forward's other stage (all layers).
+dbf_status launch_decode_group(DecodeGroup& group, int64_t peer_rows, bool class_expand, bool out_f32,
+                               const DeviceInfo& dev, cudaStream_t stream);
+
 dbf_status launch_prefill_gemm(const PrefillArgs& args, const __half* act, int64_t act_rows, bool out_f32,
                                const DeviceInfo& dev, cudaStream_t stream);
 

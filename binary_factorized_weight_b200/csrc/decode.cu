@@ -114,14 +114,21 @@ __host__ __device__ inline DecSmem dec_smem_layout(int piece, int nvalid, int nt
 
 // One launch computes RT*16 rows per CTA.  Its 4 warps form RT row tiles x
 // KW = 4/RT K slices; a cluster of ks CTAs along K splits the reduction further.
+// The launch may cover several layers that share their input (a group): the
+// CTA's tile index picks its layer.
 template <int NT, int RT, bool CLASS, bool KSCALE, bool OUT_F32>
-__global__ void __launch_bounds__(kDecThreads, 1) dbf_decode_stage_kernel(const DecodeArgs p, const int piece) {
+__global__ void __launch_bounds__(kDecThreads, 1)
+    dbf_decode_stage_kernel(const __grid_constant__ DecodeGroup grp, const int piece) {
   constexpr int NTOK = NT * 8;
   constexpr int NACC = CLASS ? 16 : 4;
   constexpr int D = kGroupBlocks;
   constexpr int KW = 4 / RT;
   constexpr int ROWS = RT * 16;
   extern __shared__ __align__(128) uint8_t smem[];
+
+  int li = 0;
+  while (li + 1 < grp.n && static_cast<int>(blockIdx.x) >= grp.tile_start[li + 1]) ++li;
+  const DecodeArgs& p = grp.layer[li];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -144,7 +151,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dbf_decode_stage_kernel(const 
   const int warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const int rt = warp / KW, kw = warp % KW;
-  const int m0 = blockIdx.x * ROWS;
+  const int m0 = (static_cast<int>(blockIdx.x) - grp.tile_start[li]) * ROWS;
   const int row0 = m0 + rt * 16 + g;
   const int k_lo = rank * p.kchunk;
   const int k_hi = min(p.K, k_lo + p.kchunk);
@@ -176,7 +183,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) dbf_decode_stage_kernel(const 
   auto load_static = [&](int pk, int pe) {
     if (tid < ROWS) rs_s[tid] = (m0 + tid < p.M) ? __half2float(p.rowscale[m0 + tid]) : 0.f;
     if constexpr (KSCALE) {
-      if (tid == 0) {
+      if (tid == 0 && pe > pk) {
         const uint32_t bytes = static_cast<uint32_t>(pe - pk) * 2;
         mbar_arrive_expect_tx(bar_b, bytes);
         bulk_load(b_s, p.kscale + pk, bytes, bar_b);
@@ -233,7 +240,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) dbf_decode_stage_kernel(const 
 
   bool ok = true;
   uint32_t phase = 0;
-  for (;;) {
+  // In a group, a layer whose K is shorter than the launch's split may leave a
+  // rank without columns; its partial sums are zero.
+  const bool has_k = k_lo < k_hi;
+  while (has_k) {
     const int plen = pe - pk;  // multiple of 64
     // ---- bring the activation rows of this piece into shared memory
     if (tid == 0) {
@@ -415,15 +425,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) dbf_decode_stage_kernel(const 
 }
 
 template <int NT, int RT, bool CLASS, bool KSCALE, bool OUT_F32>
-dbf_status launch_typed(const DecodeArgs& a, int ks, int piece, cudaStream_t stream) {
+dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cudaStream_t stream) {
   auto kernel = dbf_decode_stage_kernel<NT, RT, CLASS, KSCALE, OUT_F32>;
-  const DecSmem L = dec_smem_layout(piece, a.batch < NT * 8 ? a.batch : NT * 8, NT * 8, ks, RT);
+  const DecSmem L = dec_smem_layout(piece, batch < NT * 8 ? batch : NT * 8, NT * 8, ks, RT);
   const size_t smem = static_cast<size_t>(L.total);
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return DBF_ERR_CUDA;
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((a.M + RT * 16 - 1) / (RT * 16)), static_cast<unsigned>(ks), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(grp.tile_start[grp.n]), static_cast<unsigned>(ks), 1);
   cfg.blockDim = dim3(kDecThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -436,23 +446,23 @@ dbf_status launch_typed(const DecodeArgs& a, int ks, int piece, cudaStream_t str
   attrs[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
-  err = cudaLaunchKernelEx(&cfg, kernel, a, piece);
+  err = cudaLaunchKernelEx(&cfg, kernel, grp, piece);
   return err == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
 template <int NT, int RT>
-dbf_status launch_rt(const DecodeArgs& a, bool class_expand, bool out_f32, int ks, int piece, cudaStream_t stream) {
-  const bool kscale = a.kscale != nullptr;
+dbf_status launch_rt(const DecodeGroup& g, int batch, bool kscale, bool class_expand, bool out_f32, int ks, int piece,
+                     cudaStream_t stream) {
   if (class_expand) {
-    if (kscale) return out_f32 ? launch_typed<NT, RT, true, true, true>(a, ks, piece, stream)
-                               : launch_typed<NT, RT, true, true, false>(a, ks, piece, stream);
-    return out_f32 ? launch_typed<NT, RT, true, false, true>(a, ks, piece, stream)
-                   : launch_typed<NT, RT, true, false, false>(a, ks, piece, stream);
+    if (kscale) return out_f32 ? launch_typed<NT, RT, true, true, true>(g, batch, ks, piece, stream)
+                               : launch_typed<NT, RT, true, true, false>(g, batch, ks, piece, stream);
+    return out_f32 ? launch_typed<NT, RT, true, false, true>(g, batch, ks, piece, stream)
+                   : launch_typed<NT, RT, true, false, false>(g, batch, ks, piece, stream);
   }
-  if (kscale) return out_f32 ? launch_typed<NT, RT, false, true, true>(a, ks, piece, stream)
-                             : launch_typed<NT, RT, false, true, false>(a, ks, piece, stream);
-  return out_f32 ? launch_typed<NT, RT, false, false, true>(a, ks, piece, stream)
-                 : launch_typed<NT, RT, false, false, false>(a, ks, piece, stream);
+  if (kscale) return out_f32 ? launch_typed<NT, RT, false, true, true>(g, batch, ks, piece, stream)
+                             : launch_typed<NT, RT, false, true, false>(g, batch, ks, piece, stream);
+  return out_f32 ? launch_typed<NT, RT, false, false, true>(g, batch, ks, piece, stream)
+                 : launch_typed<NT, RT, false, false, false>(g, batch, ks, piece, stream);
 }
 
 }  // namespace
@@ -499,13 +509,38 @@ static DecodePlan plan_decode(int64_t M, int64_t K, int batch, int num_sms, int6
   return DecodePlan{4, ks_eff, piece, kchunk};
 }
 
-dbf_status launch_decode_stage(const DecodeArgs& args_in, bool class_expand, bool out_f32, const DeviceInfo& dev,
+dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_expand, bool out_f32,
+                               const DeviceInfo& dev, cudaStream_t stream) {
+  if (grp.n < 1 || grp.n > kMaxGroup) return DBF_ERR_INVALID_ARG;
+  const int batch = grp.layer[0].batch;
+  const bool kscale = grp.layer[0].kscale != nullptr;
+  int64_t tiles = 0, k_max = 0;
+  for (int g = 0; g < grp.n; ++g) {
+    const DecodeArgs& l = grp.layer[g];
+    if (l.batch != batch || (l.kscale != nullptr) != kscale) return DBF_ERR_INVALID_ARG;
+    grp.tile_start[g] = static_cast<int>(tiles);
+    tiles += (l.M + 63) / 64;
+    k_max = std::max<int64_t>(k_max, l.K);
+  }
+  if (tiles > 0x7fffffffLL) return DBF_ERR_UNSUPPORTED_SHAPE;
+  grp.tile_start[grp.n] = static_cast<int>(tiles);
+  // one K split for the launch, planned for its rows and its longest K; every
+  // layer cuts its own K into that many 256-column-aligned chunks
+  const DecodePlan plan = plan_decode(64 * tiles, k_max, batch, dev.num_sms, peer_rows);
+  for (int g = 0; g < grp.n; ++g) {
+    int64_t kc = (grp.layer[g].K + plan.ks - 1) / plan.ks;
+    grp.layer[g].kchunk = static_cast<int>((kc + 255) / 256 * 256);
+  }
+  if (batch > 8) return launch_rt<2, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+  return launch_rt<1, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+}
+
+dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
                                cudaStream_t stream) {
-  DecodeArgs a = args_in;
-  const DecodePlan plan = plan_decode(a.M, a.K, a.batch, dev.num_sms, a.peer_rows);
-  a.kchunk = static_cast<int>(plan.kchunk);
-  if (a.batch > 8) return launch_rt<2, 4>(a, class_expand, out_f32, plan.ks, plan.piece, stream);
-  return launch_rt<1, 4>(a, class_expand, out_f32, plan.ks, plan.piece, stream);
+  DecodeGroup grp{};
+  grp.n = 1;
+  grp.layer[0] = args;
+  return launch_decode_group(grp, args.peer_rows, class_expand, out_f32, dev, stream);
 }
 
 }  // namespace dbf

@@ -204,6 +204,48 @@ DBF_API dbf_status dbf_forward_noalloc(const uint16_t* x, const uint32_t* packed
                                        int64_t k, int64_t m_in, int64_t batch, void* y, dbf_dtype y_t,
                                        uint32_t flags, struct CUstream_st* stream);
 
+/*
+ * Several layers that read the same input x: the same computation as one
+ * dbf_forward per layer (section 2.1, computation process), with the layers'
+ * first products in one launch and their second products in another.  The
+ * pages evaluate one layer at a time; grouping layers that share their input
+ * (a decoder's q, k and v projections, or its gate and up projections) is an
+ * engineering choice of this library: at batch 1 each launch costs latency
+ * that does not grow with its size, so G layers in two launches cost far less
+ * than G layers in 2G.
+ *
+ *   layers[g]  packedA, packedB, a, m, b: as in dbf_forward for layer g, of
+ *              n = layers[g].n rows and middle dimension k = layers[g].k, all
+ *              over the shared m_in; y: batch x n output of layer g
+ *              (row-major, y_t).  The array is read during the call only.
+ *   num_layers 1 .. DBF_MAX_GROUP.
+ *   workspace  ws_bytes >= dbf_forward_grouped_workspace_bytes(...) for the
+ *              same layers, zero-filled before its first use.
+ * Per-layer results equal dbf_forward's up to the order of fp32 additions
+ * (the K split can differ); in integer mode they are identical.
+ * Shape contract per layer as dbf_forward; flags as dbf_forward.
+ */
+#define DBF_MAX_GROUP 8
+typedef struct dbf_layer_desc {
+  const uint32_t* packedA;
+  const uint32_t* packedB;
+  const uint16_t* a;
+  const uint16_t* m;
+  const uint16_t* b;
+  int64_t n;
+  int64_t k;
+  void* y;
+} dbf_layer_desc;
+
+/* Workspace bytes for dbf_forward_grouped (0 if an argument is out of range):
+ * 256 + sum over layers of round_up(batch * k_g * 2, 256). */
+DBF_API size_t dbf_forward_grouped_workspace_bytes(const dbf_layer_desc* layers, int num_layers, int64_t m_in,
+                                                   int64_t batch);
+
+DBF_API dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, const dbf_layer_desc* layers,
+                                       int num_layers, dbf_dtype y_t, void* workspace, size_t ws_bytes,
+                                       uint32_t flags, struct CUstream_st* stream);
+
 /* Static, NUL-terminated description of a status code. */
 DBF_API const char* dbf_status_string(dbf_status status);
 

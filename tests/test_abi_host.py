@@ -138,3 +138,48 @@ def test_workspace_status_validation(lib):
     out = ctypes.c_int32()
     assert lib.dbf_workspace_status(None, None, ctypes.byref(out)) == INVALID
     assert lib.dbf_workspace_status(P, None, None) == INVALID
+
+
+def grouped(lib, descs=None, x=P, m_in=256, batch=4, y_t=1, ws=P, ws_bytes=1 << 20, flags=0, num=None):
+    if descs is None:
+        descs = [dict(n=256, k=128), dict(n=64, k=64)]
+    arr = (dbf._LayerDesc * max(1, len(descs)))()
+    for i, d in enumerate(descs):
+        arr[i] = dbf._LayerDesc(d.get("A", P), d.get("B", P), d.get("a", P), d.get("m", P), d.get("b", P),
+                                d.get("n", 256), d.get("k", 128), d.get("y", P))
+    return lib.dbf_forward_grouped(x, m_in, batch, arr, len(descs) if num is None else num, y_t, ws, ws_bytes,
+                                   flags, None)
+
+
+def test_grouped_workspace_bytes(lib):
+    # 256 + sum of round_up(batch * k_g * 2, 256)
+    assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=256, k=128), dict(n=64, k=64)], 256, 4) == \
+        256 + 1024 + 512
+    assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=8, k=832)], 4096, 3) == 256 + 5120
+    assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=0, k=64)], 64, 1) == 0
+    assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=1, k=64)] * 9, 64, 1) == 0
+
+
+@pytest.mark.parametrize(
+    "kwargs,expect",
+    [
+        (dict(x=None), INVALID), (dict(num=0), INVALID), (dict(num=9), INVALID),
+        (dict(descs=[dict(y=None)]), INVALID), (dict(descs=[dict(A=None)]), INVALID),
+        (dict(descs=[dict(n=0)]), INVALID), (dict(descs=[dict(k=96)]), SHAPE), (dict(m_in=100), SHAPE),
+        (dict(descs=[dict(), dict(k=1 << 21)]), SHAPE),
+        (dict(batch=0), INVALID), (dict(y_t=2 + 5), INVALID), (dict(flags=2 | 4), INVALID),
+        (dict(x=MIS), MISALIGNED), (dict(descs=[dict(), dict(y=MIS)]), MISALIGNED),
+        (dict(descs=[dict(B=MIS)]), MISALIGNED),
+        (dict(ws=None), WORKSPACE), (dict(ws_bytes=256 + 1024 + 511), WORKSPACE),
+    ],
+)
+def test_grouped_validation(lib, kwargs, expect):
+    assert grouped(lib, **kwargs) == expect
+
+
+def test_grouped_valid_args_without_device(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; covered by the gpu tests")
+    assert grouped(lib) in (CUDA_ERR, 7)
