@@ -35,6 +35,8 @@ def _setup(lib):
     lib.oracle_pack_signs.restype = None
     lib.oracle_forward_staged.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, vp]
     lib.oracle_forward_staged.restype = None
+    lib.oracle_forward_transposed.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.oracle_forward_transposed.restype = None
     lib.oracle_dense_weight.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     lib.oracle_dense_weight.restype = None
     lib.oracle_forward_dense.argtypes = [vp, vp, i64, i64, i64, vp]
@@ -133,6 +135,26 @@ def forward_staged(x, A, B, a, mid, b, return_v: bool = False):
     lib.oracle_forward_staged(_ptr(x), _ptr(A), _ptr(B), _ptr(a), _ptr(mid), _ptr(b), n, k, m_in,
                               batch, _ptr(y), _ptr(v) if v is not None else None)
     return (y, v) if return_v else y
+
+
+def forward_transposed(dy, A, B, a, mid, b):
+    """dx = dy W for W = (a (.) A (.) mid^T)(B (.) b^T), fp64, right to left without forming W
+    (the transpose of the forward of section 2.1).  dy: batch x n; returns batch x m_in."""
+    lib = _load()
+    dy = _f64(dy)
+    if dy.ndim == 1:
+        dy = dy[None, :]
+    A, B = _i8(A), _i8(B)
+    a, mid, b = _f64(a), _f64(mid), _f64(b)
+    n, k = A.shape
+    k2, m_in = B.shape
+    batch = dy.shape[0]
+    if k2 != k or dy.shape[1] != n or a.size != n or mid.size != k or b.size != m_in:
+        raise ValueError("shape mismatch")
+    dx = np.empty((batch, m_in), dtype=np.float64)
+    lib.oracle_forward_transposed(_ptr(dy), _ptr(A), _ptr(B), _ptr(a), _ptr(mid), _ptr(b), n, k, m_in, batch,
+                                  _ptr(dx))
+    return dx
 
 
 def dense_weight(A, B, a, mid, b) -> np.ndarray:

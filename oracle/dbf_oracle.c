@@ -143,6 +143,43 @@ void oracle_forward_staged(const double* x, const int8_t* A, const int8_t* B, co
   free(vbuf);
 }
 
+/* The transpose product dx = dy W for the factorised W (section 2.1: W is
+ * n x m_in with y = x W^T, so dy W is the product with W^T's transpose, the
+ * input gradient of the layer).  With W = (a (.) A (.) mid^T)(B (.) b^T):
+ *     dx[t][j] = b_j * sum_l B[l][j] * mid_l * sum_i A[i][l] * a_i * dy[t][i],
+ * evaluated right to left like the forward, without forming W.
+ * dy: batch x n; dx: batch x m_in.  fp64 throughout. */
+void oracle_forward_transposed(const double* dy, const int8_t* A, const int8_t* B, const double* a,
+                               const double* mid, const double* b, int64_t n, int64_t k, int64_t m_in,
+                               int64_t batch, double* dx) {
+  double* gbuf = (double*)malloc((size_t)n * sizeof(double));
+  double* vbuf = (double*)malloc((size_t)k * sizeof(double));
+  if (!gbuf || !vbuf) {
+    free(gbuf);
+    free(vbuf);
+    for (int64_t e = 0; e < batch * m_in; ++e) dx[e] = NAN;
+    return;
+  }
+  for (int64_t tok = 0; tok < batch; ++tok) {
+    const double* dyt = dy + tok * n;
+    for (int64_t i = 0; i < n; ++i) gbuf[i] = a[i] * dyt[i];
+#pragma omp parallel for schedule(static)
+    for (int64_t l = 0; l < k; ++l) {
+      double acc = 0.0;
+      for (int64_t i = 0; i < n; ++i) acc += (double)A[i * k + l] * gbuf[i];
+      vbuf[l] = mid[l] * acc;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < m_in; ++j) {
+      double acc = 0.0;
+      for (int64_t l = 0; l < k; ++l) acc += (double)B[l * m_in + j] * vbuf[l];
+      dx[tok * m_in + j] = b[j] * acc;
+    }
+  }
+  free(gbuf);
+  free(vbuf);
+}
+
 /*
  * Dense reconstruction W = (a (.) A (.) m^T)(B (.) b^T), n x m_in:
  *   W[i][j] = sum_l (a_i A[i][l] m_l) (B[l][j] b_j)

@@ -1,7 +1,8 @@
 """Plant plausible mistakes in copies of the oracle and check the pins catch each.
 
 Each mutant is the oracle's C source with one edit (a dropped scale, a wrong
-sign, a transposed or reversed operand, a dropped term, a wrong bit layout),
+sign, a transposed or reversed operand, a dropped term, a wrong bit layout,
+in the forward and in the transpose product),
 compiled into a temporary library on the CPU.  The pins of
 test_oracle_pins.py are then run against the mutant; at least one must fail.
 This shows the pins are strong enough to trust the unmutated oracle.
@@ -34,6 +35,13 @@ MUTANTS = {
     "dense_drops_b": ("Wi[j] += left * ((double)Bl[j] * b[j]);", "Wi[j] += left * ((double)Bl[j]);"),
     "dense_transposed_B": ("Wi[j] += left * ((double)Bl[j] * b[j]);",
                            "Wi[j] += left * ((double)B[(j % k) * m_in + (l % m_in)] * b[j]);"),
+    "transposed_drops_b": ("dx[tok * m_in + j] = b[j] * acc;", "dx[tok * m_in + j] = acc;"),
+    "transposed_scales_swapped": ("for (int64_t i = 0; i < n; ++i) gbuf[i] = a[i] * dyt[i];",
+                                  "for (int64_t i = 0; i < n; ++i) gbuf[i] = a[(i + 1) % n] * dyt[i];"),
+    "transposed_reads_A_as_k_by_n": ("acc += (double)A[i * k + l] * gbuf[i];",
+                                     "acc += (double)A[l * n + i] * gbuf[i];"),
+    "transposed_B_not_transposed": ("acc += (double)B[l * m_in + j] * vbuf[l];",
+                                    "acc += (double)B[(j % k) * m_in + (l % m_in)] * vbuf[l];"),
     "bpw_off": ("return (double)k * (double)(n + m_in) / ((double)n * (double)m_in);",
                 "return (double)k * (double)(n + m_in) / ((double)n * (double)(m_in + 1));"),
 }
@@ -51,6 +59,11 @@ PIN_CHECKS = [
     lambda o: pins.test_layout_table(o),
     lambda o: pins.test_layout_round_trip_and_padding(o, 3, 128),
     lambda o: pins.test_layout_hand_words(o),
+    lambda o: pins.test_transposed_adjoint_identity(o, 48, 64, 80, 3),
+    lambda o: pins.test_transposed_equals_dense(o, 33, 64, 65, 3),
+    lambda o: pins.test_transposed_hadamard_closed_form(o, 3),
+    lambda o: pins.test_transposed_integer_exact(o),
+    lambda o: pins.test_transposed_uses_each_scale_once(o),
 ]
 
 

@@ -319,3 +319,76 @@ def test_layout_round_trip_and_padding(oracle_mod, rows, cols):
         corrupt = packed.copy()
         corrupt[wpr - 1] |= np.uint32(1 << 31)  # group 15, pair 7, odd: column 255 of the last block
         assert oracle_mod.unpack_signs(corrupt, rows, cols)[1] == 1
+
+
+# ---------------------------------------------------------------- the transpose product dx = dy W
+@pytest.mark.parametrize("n,k,m_in,batch", [(48, 64, 80, 3), (7, 5, 11, 2)])
+def test_transposed_adjoint_identity(oracle_mod, n, k, m_in, batch):
+    """<y(x), dy> = <x, dx(dy)> for every x and dy: the defining property of the transpose."""
+    rng = np.random.default_rng(7 * n + k)
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    a, mid, b = gen.lognormal_scales(rng, n), gen.abs_normal_scales(rng, k), gen.lognormal_scales(rng, m_in)
+    x = gen.normal_activations(rng, batch, m_in).astype(np.float64)
+    dy = gen.normal_activations(rng, batch, n).astype(np.float64)
+    lhs = np.sum(oracle_mod.forward_staged(x, A, B, a, mid, b) * dy)
+    rhs = np.sum(x * oracle_mod.forward_transposed(dy, A, B, a, mid, b))
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+
+
+@pytest.mark.parametrize("n,k,m_in,batch", [(96, 64, 320, 2), (33, 64, 65, 3)])
+def test_transposed_equals_dense(oracle_mod, n, k, m_in, batch):
+    """dx = dy W against numpy's matmul with the dense factors written out here."""
+    rng = np.random.default_rng(n * k + m_in)
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    a, mid, b = gen.abs_normal_scales(rng, n), gen.lognormal_scales(rng, k), gen.abs_normal_scales(rng, m_in)
+    dy = gen.normal_activations(rng, batch, n).astype(np.float64)
+    W_np = (a.astype(np.float64)[:, None] * A * mid.astype(np.float64)[None, :]) @ (B * b.astype(np.float64)[None, :])
+    dx = oracle_mod.forward_transposed(dy, A, B, a, mid, b)
+    assert np.linalg.norm(dx - dy @ W_np) <= 1e-12 * np.linalg.norm(dx)
+
+
+@pytest.mark.parametrize("p", [3, 5])
+def test_transposed_hadamard_closed_form(oracle_mod, p):
+    """A = B = H (symmetric): dx = b (.) FWHT(mid (.) FWHT(a (.) dy))."""
+    size = 1 << p
+    H = gen.sylvester_hadamard(p)
+    rng = np.random.default_rng(100 + p)
+    a, mid, b = gen.abs_normal_scales(rng, size), gen.lognormal_scales(rng, size), gen.lognormal_scales(rng, size)
+    dy = gen.normal_activations(rng, 2, size).astype(np.float64)
+    dx = oracle_mod.forward_transposed(dy, H, H, a, mid, b)
+    closed = b.astype(np.float64) * _fwht(mid.astype(np.float64) * _fwht(a.astype(np.float64) * dy))
+    assert np.allclose(dx, closed, rtol=1e-12, atol=1e-12 * np.abs(closed).max())
+
+
+def test_transposed_integer_exact(oracle_mod):
+    """Unit scales, integer dy: dx equals the int64 product dy A B."""
+    rng = np.random.default_rng(3)
+    n, k, m_in = 40, 24, 56
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    dy = rng.integers(-8, 9, size=(3, n))
+    ones = lambda s: np.ones(s, dtype=np.float16)
+    dx = oracle_mod.forward_transposed(dy, A, B, ones(n), ones(k), ones(m_in))
+    exact = dy.astype(np.int64) @ A.astype(np.int64) @ B.astype(np.int64)
+    assert np.array_equal(dx, exact.astype(np.float64))
+
+
+def test_transposed_uses_each_scale_once(oracle_mod):
+    """One-hot scales pick single entries: dx[j] = b_j * B[l, j] * mid_l * A[i, l] * a_i * dy[i]."""
+    rng = np.random.default_rng(11)
+    n, k, m_in = 6, 4, 5
+    A = gen.sign_matrix(rng, n, k)
+    B = gen.sign_matrix(rng, k, m_in)
+    i, l = 2, 1
+    a = np.zeros(n, dtype=np.float16)
+    a[i] = 3
+    mid = np.zeros(k, dtype=np.float16)
+    mid[l] = 5
+    b = np.arange(1, m_in + 1).astype(np.float16)
+    dy = np.zeros((1, n))
+    dy[0, i] = 2
+    dx = oracle_mod.forward_transposed(dy, A, B, a, mid, b)
+    expect = b.astype(np.float64) * B[l].astype(np.float64) * 5 * A[i, l] * 3 * 2
+    assert np.array_equal(dx[0], expect)
