@@ -274,6 +274,29 @@ class Workload:
         return g
 
 
+class TransposedWorkload(Workload):
+    """The same R layer copies run as the transpose product dx = dy W (dy: batch x n)."""
+
+    def __init__(self, dbf, torch, shape, batch, device, copies=None):
+        super().__init__(dbf, torch, shape, batch, device, copies=copies)
+        n, k, m_in = shape.n, shape.k, shape.m_in
+        self.pAT = [dbf.dbf_transpose_signs(pA, n, k) for pA in self.pA]
+        self.pBT = [dbf.dbf_transpose_signs(pB, k, m_in) for pB in self.pB]
+        rng = np.random.default_rng(7)
+        self.dy = torch.from_numpy(gen.normal_activations(rng, batch, n)).to(device)
+        self.dx = torch.empty((batch, m_in), dtype=torch.float16, device=device)
+        self.ws = dbf.dbf_new_workspace(m_in, k, n, batch, device=device)
+        self.bytes = layer_bytes(m_in, k, n, batch)
+        self.path = "transposed " + self.path
+
+    def forward_all(self, x=None, y=None):
+        s = self.shape
+        for i in range(self.copies):
+            a, mid, b = self.sc[i]
+            self.dbf.dbf_forward_transposed(self.dy, self.pAT[i], self.pBT[i], a, mid, b, s.n, s.k, s.m_in,
+                                            dx=self.dx, workspace=self.ws, flags=self.flags)
+
+
 GROUPS = {"qkv": ("q", "k", "v"), "gate_up": ("gate", "up")}
 
 
@@ -553,6 +576,35 @@ def run_sweep(args):
                "tensor_frac": tf / peaks["bf16_tflops"], "copies": wl.copies, "path": wl.path,
                "context_torch_fp16_dense_us": dense_us,
                "speedup_vs_dense_fp16": dense_us / us}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        del g, wl
+        torch.cuda.empty_cache()
+    # the transpose product dx = dy W on the same layers
+    for shape, batch in [(gen.CONFIGS["attn_1b"], 1), (gen.CONFIGS["attn_1b"], 2048), (gen.CONFIGS["mlp_up"], 1),
+                         (gen.CONFIGS["mlp_up"], 2048)]:
+        wl = TransposedWorkload(dbf, torch, shape, batch, device)
+        g = wl.capture()
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+        reps = max(3, int(200 / max(1, wl.copies)))
+        times = []
+        for _ in range(7):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / reps / wl.copies * 1e3)
+        us = statistics.median(times)
+        gbs = wl.bytes / (us * 1e-6) / 1e9
+        tf = layer_flops(shape.n, shape.k, shape.m_in, batch) / (us * 1e-6) / 1e12
+        row = {"layer": f"{shape.name} (transposed: dx = dy W)", "n": shape.n, "k": shape.k, "m_in": shape.m_in,
+               "batch": batch, "us": us, "us_p10": sorted(times)[0], "us_p90": sorted(times)[-1],
+               "tokens_per_s": batch / (us * 1e-6), "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": tf,
+               "tensor_frac": tf / peaks["bf16_tflops"], "copies": wl.copies, "path": wl.path}
         rows.append(row)
         print(json.dumps(row), flush=True)
         del g, wl

@@ -31,6 +31,7 @@ __all__ = [
     "dbf_forward_workspace_bytes", "dbf_new_workspace", "dbf_forward",
     "dbf_reconstruct_dense", "dbf_workspace_status", "dbf_status_string", "dbf_forward_noalloc",
     "DBF_MAX_GROUP", "dbf_forward_grouped_workspace_bytes", "dbf_new_grouped_workspace", "dbf_forward_grouped",
+    "dbf_transpose_signs", "dbf_forward_transposed",
 ]
 
 DBF_I8, DBF_F16, DBF_F32 = 0, 1, 2
@@ -55,6 +56,8 @@ EXPORTED_SYMBOLS = (
     "dbf_forward_noalloc",
     "dbf_forward_grouped_workspace_bytes",
     "dbf_forward_grouped",
+    "dbf_transpose_signs",
+    "dbf_forward_transposed",
     "dbf_status_string",
 )
 
@@ -113,6 +116,10 @@ def load_library():
     lib.dbf_forward_grouped_workspace_bytes.restype = sz
     lib.dbf_forward_grouped.argtypes = [vp, i64, i64, ctypes.POINTER(_LayerDesc), i32, i32, vp, sz, u32, vp]
     lib.dbf_forward_grouped.restype = i32
+    lib.dbf_transpose_signs.argtypes = [vp, i64, i64, vp, vp]
+    lib.dbf_transpose_signs.restype = i32
+    lib.dbf_forward_transposed.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, vp, sz, u32, vp]
+    lib.dbf_forward_transposed.restype = i32
     lib.dbf_status_string.argtypes = [i32]
     lib.dbf_status_string.restype = ctypes.c_char_p
     _LIB = lib
@@ -284,3 +291,37 @@ def dbf_forward_grouped(x: torch.Tensor, layers, m_in: int, ys=None, y_dtype: to
         _ptr(x), int(m_in), int(batch), arr, len(layers), _dtype_code(ys[0].dtype), _ptr(workspace),
         workspace.numel() * workspace.element_size(), int(flags), _stream(stream)))
     return ys
+
+
+def dbf_transpose_signs(packed: torch.Tensor, rows: int, cols: int, out: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """Packed S (rows x cols) -> packed S^T (cols x rows), int32 CUDA tensor."""
+    n_words = dbf_packed_words(cols, rows)
+    if out is None:
+        out = torch.empty(n_words, dtype=torch.int32, device=packed.device)
+    elif out.numel() < n_words or out.dtype != torch.int32:
+        raise ValueError("out must be an int32 tensor of dbf_packed_words(cols, rows) words")
+    _check("dbf_transpose_signs", load_library().dbf_transpose_signs(
+        _ptr(packed), int(rows), int(cols), _ptr(out), _stream(stream)))
+    return out
+
+
+def dbf_forward_transposed(dy: torch.Tensor, packedAT: torch.Tensor, packedBT: torch.Tensor, a: torch.Tensor,
+                           m: torch.Tensor, b: torch.Tensor, n: int, k: int, m_in: int, dx: Optional[torch.Tensor] = None,
+                           dx_dtype: torch.dtype = torch.float16, workspace: Optional[torch.Tensor] = None,
+                           flags: int = 0, stream=None) -> torch.Tensor:
+    """dx = b (.) (B^T (m (.) (A^T (a (.) dy)))) for fp16 dy (batch x n); returns dx (batch x m_in)."""
+    if dy.dtype != torch.float16 or dy.dim() != 2 or not dy.is_contiguous():
+        raise ValueError("dy must be a contiguous fp16 batch x n tensor")
+    batch = dy.shape[0]
+    if dy.shape[1] != n:
+        raise ValueError("dy.shape[1] != n")
+    if dx is None:
+        dx = torch.empty((batch, m_in), dtype=dx_dtype, device=dy.device)
+    if workspace is None:
+        workspace = dbf_new_workspace(m_in, k, n, batch, device=dy.device)
+    _check("dbf_forward_transposed", load_library().dbf_forward_transposed(
+        _ptr(dy), _ptr(packedAT), _ptr(packedBT), _ptr(a), _ptr(m), _ptr(b), int(n), int(k), int(m_in), int(batch),
+        _ptr(dx), _dtype_code(dx.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(), int(flags),
+        _stream(stream)))
+    return dx

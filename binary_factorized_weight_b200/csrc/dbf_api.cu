@@ -343,6 +343,31 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
   return DBF_OK;
 }
 
+dbf_status dbf_transpose_signs(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out,
+                               struct CUstream_st* stream) {
+  if (!packed || !out) return DBF_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1) return DBF_ERR_INVALID_ARG;
+  if (rows > kMaxRows || cols > kMaxRows || rows * words_per_row(cols) > (int64_t{1} << 40) ||
+      cols * words_per_row(rows) > (int64_t{1} << 40))
+    return DBF_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(packed) || !aligned16(out)) return DBF_ERR_MISALIGNED;
+  DeviceInfo dev;
+  dbf_status st = current_device(&dev);
+  if (st != DBF_OK) return st;
+  return launch_transpose_signs(packed, rows, cols, out, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dbf_status dbf_forward_transposed(const uint16_t* dy, const uint32_t* packedAT, const uint32_t* packedBT,
+                                  const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n, int64_t k,
+                                  int64_t m_in, int64_t batch, void* dx, dbf_dtype dx_t, void* workspace,
+                                  size_t ws_bytes, uint32_t flags, struct CUstream_st* stream) {
+  // dx = b (.) (B^T (m (.) (A^T (a (.) dy)))): the forward with B^T (m_in rows
+  // over k) as its first factor and A^T (k rows over n) as its second, a and b
+  // exchanged, and n in the place of m_in.
+  return dbf_forward(dy, packedBT, packedAT, b, m, a, m_in, k, n, batch, dx, dx_t, workspace, ws_bytes, flags,
+                     stream);
+}
+
 dbf_status dbf_reconstruct_dense(const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
                                  const uint16_t* m, const uint16_t* b, int64_t n, int64_t k, int64_t m_in, void* W,
                                  dbf_dtype W_t, struct CUstream_st* stream) {

@@ -79,6 +79,9 @@ dbf_status launch_prefill_gemm(const PrefillArgs& args, const __half* act, int64
 dbf_status launch_pack(const void* src, dbf_dtype src_t, int64_t rows, int64_t cols, uint32_t* packed,
                        const DeviceInfo& dev, cudaStream_t stream);
 
+dbf_status launch_transpose_signs(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out,
+                                  const DeviceInfo& dev, cudaStream_t stream);
+
 dbf_status launch_reconstruct(const uint32_t* packedA, const uint32_t* packedB, const __half* a, const __half* mid,
                               const __half* b, int64_t n, int64_t k, int64_t m_in, void* W, bool out_f32,
                               const DeviceInfo& dev, cudaStream_t stream);

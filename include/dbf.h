@@ -246,6 +246,38 @@ DBF_API dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t 
                                        int num_layers, dbf_dtype y_t, void* workspace, size_t ws_bytes,
                                        uint32_t flags, struct CUstream_st* stream);
 
+/*
+ * Transpose of a packed sign matrix: `packed` holds S (rows x cols) in the
+ * packed layout; `out` receives S^T (cols rows over `rows` columns), i.e.
+ * dbf_packed_words(cols, rows) words, in the same layout with zero padding.
+ * Used to pack A^T and B^T for dbf_forward_transposed without the +-1 matrices.
+ * Not a hot path.  Both pointers 16-byte aligned; out must not overlap packed.
+ */
+DBF_API dbf_status dbf_transpose_signs(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out,
+                                       struct CUstream_st* stream);
+
+/*
+ * The transpose product dx = dy W of the layer of dbf_forward (W is n x m_in,
+ * y = x W^T, so this is the input gradient):
+ *     dx = b (.) (B^T (m (.) (A^T (a (.) dy))))      (section 2.1 read right to left)
+ *   dy         batch x n fp16, row-major.
+ *   packedAT   A^T packed: k rows over n   (dbf_transpose_signs of packedA).
+ *   packedBT   B^T packed: m_in rows over k (dbf_transpose_signs of packedB).
+ *   a, m, b    the layer's scales (n, k, m_in entries), as in dbf_forward.
+ *   dx         batch x m_in, dx_t = DBF_F16 or DBF_F32.
+ *   workspace  ws_bytes >= dbf_forward_workspace_bytes(m_in, k, n, batch).
+ * It is dbf_forward with B^T and A^T as the two factors and a and b
+ * exchanged, so the arithmetic (fp32 accumulation, fp16 a (.) dy on the decode
+ * path, fp16 middle vector) and the paths are those of dbf_forward.  Shape
+ * contract: k and n multiples of 64 in [64, 1 << 20], m_in and batch in
+ * [1, 1 << 24].
+ */
+DBF_API dbf_status dbf_forward_transposed(const uint16_t* dy, const uint32_t* packedAT, const uint32_t* packedBT,
+                                          const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n,
+                                          int64_t k, int64_t m_in, int64_t batch, void* dx, dbf_dtype dx_t,
+                                          void* workspace, size_t ws_bytes, uint32_t flags,
+                                          struct CUstream_st* stream);
+
 /* Static, NUL-terminated description of a status code. */
 DBF_API const char* dbf_status_string(dbf_status status);
 

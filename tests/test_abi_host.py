@@ -183,3 +183,24 @@ def test_grouped_valid_args_without_device(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present; covered by the gpu tests")
     assert grouped(lib) in (CUDA_ERR, 7)
+
+
+def test_transpose_validation(lib):
+    assert lib.dbf_transpose_signs(None, 4, 64, P, None) == INVALID
+    assert lib.dbf_transpose_signs(P, 4, 64, None, None) == INVALID
+    assert lib.dbf_transpose_signs(P, 0, 64, P, None) == INVALID
+    assert lib.dbf_transpose_signs(P, 4, (1 << 24) + 1, P, None) == SHAPE
+    assert lib.dbf_transpose_signs(MIS, 4, 64, P, None) == MISALIGNED
+    assert lib.dbf_transpose_signs(P, 4, 64, MIS, None) == MISALIGNED
+
+
+def test_forward_transposed_validation(lib):
+    # dy (batch x n), dx (batch x m_in); n takes the place of the forward's m_in
+    def call(dy=P, n=256, k=128, m_in=200, batch=4, dx=P, ws_bytes=1 << 20):
+        return lib.dbf_forward_transposed(dy, P, P, P, P, P, n, k, m_in, batch, dx, 1, P, ws_bytes, 0, None)
+
+    assert call(dy=None) == INVALID
+    assert call(n=100) == SHAPE       # n must be a multiple of 64 here
+    assert call(k=96) == SHAPE
+    assert call(dx=MIS) == MISALIGNED
+    assert call(ws_bytes=255) == WORKSPACE
