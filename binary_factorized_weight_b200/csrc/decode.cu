@@ -258,43 +258,97 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     ok = __syncthreads_and(ok);
     if (!ok) break;
 
-    // ---- u = fp16(x (.) b) in place; class sums U_rest (all groups but 15).
-    // All 128 threads share each token's row; per-warp partial sums are added
-    // in warp order, so the result is deterministic.
-    if constexpr (KSCALE || CLASS) {
-      const int nch = plen / 8;
-      for (int tok = 0; tok < nvalid; ++tok) {
-        uint4* rowv = reinterpret_cast<uint4*>(act_s + tok * L.stride);
-        float sum = 0.f;
-        for (int ch = tid; ch < nch; ch += kDecThreads) {
-          uint4 v = rowv[ch];
-          if constexpr (KSCALE) {
-            const uint4 sb = reinterpret_cast<const uint4*>(b_s)[ch];
-            __half2* h = reinterpret_cast<__half2*>(&v);
-            const __half2* hb = reinterpret_cast<const __half2*>(&sb);
-            h[0] = __hmul2(h[0], hb[0]);
-            h[1] = __hmul2(h[1], hb[1]);
-            h[2] = __hmul2(h[2], hb[2]);
-            h[3] = __hmul2(h[3], hb[3]);
-            rowv[ch] = v;
+    // ---- u = fp16(x (.) b) in place; class sums U_rest (all groups but 15),
+    // per-warp parts added in warp order (deterministic).
+    // Up to 8 tokens: all 128 threads take each token's row in turn.
+    // 9 to 16 tokens: warp w owns tokens w, w+4, w+8, w+12; a thread scales and
+    // sums only what it owns, so a warp's tokens run side by side.
+    if constexpr (NT == 1) {
+      if constexpr (KSCALE || CLASS) {
+        const int nch = plen / 8;
+        for (int tok = 0; tok < nvalid; ++tok) {
+          uint4* rowv = reinterpret_cast<uint4*>(act_s + tok * L.stride);
+          float sum = 0.f;
+          for (int ch = tid; ch < nch; ch += kDecThreads) {
+            uint4 v = rowv[ch];
+            if constexpr (KSCALE) {
+              const uint4 sb = reinterpret_cast<const uint4*>(b_s)[ch];
+              __half2* h = reinterpret_cast<__half2*>(&v);
+              const __half2* hb = reinterpret_cast<const __half2*>(&sb);
+              h[0] = __hmul2(h[0], hb[0]);
+              h[1] = __hmul2(h[1], hb[1]);
+              h[2] = __hmul2(h[2], hb[2]);
+              h[3] = __hmul2(h[3], hb[3]);
+              rowv[ch] = v;
+            }
+            if constexpr (CLASS) {
+              if (((ch >> 1) & 15) != 15) {  // 8 columns = half a group; group = (8*ch mod 256)/16
+                const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sum += __low2float(h[q]) + __high2float(h[q]);
+              }
+            }
           }
           if constexpr (CLASS) {
-            if (((ch >> 1) & 15) != 15) {  // 8 columns = half a group; group = (8*ch mod 256)/16
-              const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) sum += __low2float(h[q]) + __high2float(h[q]);
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (lane == 0) upart_s[warp * 16 + tok] = sum;
+          }
+        }
+        __syncthreads();
+        if constexpr (CLASS) {
+          if (tid < nvalid) urest_s[tid] += (upart_s[tid] + upart_s[16 + tid]) + (upart_s[32 + tid] + upart_s[48 + tid]);
+        }
+      }
+    } else {
+      if constexpr (KSCALE || CLASS) {
+        const int nch = plen / 8;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int ch = lane; ch < nch; ch += 32) {
+          const bool rest = ((ch >> 1) & 15) != 15;  // 8 columns = half a group; group = (8*ch mod 256)/16
+          uint4 sb = make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (KSCALE) sb = reinterpret_cast<const uint4*>(b_s)[ch];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int tok = warp + 4 * j;
+            if (tok < nvalid) {
+              uint4* rowv = reinterpret_cast<uint4*>(act_s + tok * L.stride);
+              uint4 v = rowv[ch];
+              __half2* h = reinterpret_cast<__half2*>(&v);
+              if constexpr (KSCALE) {
+                const __half2* hb = reinterpret_cast<const __half2*>(&sb);
+                h[0] = __hmul2(h[0], hb[0]);
+                h[1] = __hmul2(h[1], hb[1]);
+                h[2] = __hmul2(h[2], hb[2]);
+                h[3] = __hmul2(h[3], hb[3]);
+                rowv[ch] = v;
+              }
+              if constexpr (CLASS) {
+                if (rest) {
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) sum[j] += __low2float(h[q]) + __high2float(h[q]);
+                }
+              }
             }
           }
         }
         if constexpr (CLASS) {
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-          if (lane == 0) upart_s[warp * 16 + tok] = sum;
+          for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sum[j] += __shfl_xor_sync(0xffffffffu, sum[j], off);
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (warp + 4 * j < nvalid) upart_s[warp * 16 + warp + 4 * j] = sum[j];
+          }
         }
-      }
-      __syncthreads();
-      if constexpr (CLASS) {
-        if (tid < nvalid) urest_s[tid] += (upart_s[tid] + upart_s[16 + tid]) + (upart_s[32 + tid] + upart_s[48 + tid]);
+        __syncthreads();
+        if constexpr (CLASS) {
+          // token t's sum comes from its owner warp t % 4 alone
+          if (tid < nvalid) urest_s[tid] += upart_s[(tid & 3) * 16 + tid];
+        }
       }
     }
 
