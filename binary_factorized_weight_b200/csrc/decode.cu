@@ -51,7 +51,9 @@ namespace dbf {
 namespace {
 
 constexpr int kDecThreads = 128;
-constexpr int kGroupBlocks = 4;  // 256-column blocks per register group of weights
+// 256-column blocks per register group of weights: 4, or 8 for rows of more
+// than 8 blocks per warp (long reductions stream their weights; a bigger group
+// keeps more of them in flight while the previous group is multiplied)
 constexpr int kMaxClusterK = 8;
 constexpr int kSmemBudget = 100 * 1024;
 constexpr int kHeadBytes = 512;  // mbarriers, abort flag, class sums and their per-warp parts
@@ -116,12 +118,11 @@ __host__ __device__ inline DecSmem dec_smem_layout(int piece, int nvalid, int nt
 // KW = 4/RT K slices; a cluster of ks CTAs along K splits the reduction further.
 // The launch may cover several layers that share their input (a group): the
 // CTA's tile index picks its layer.
-template <int NT, int RT, bool CLASS, bool KSCALE, bool OUT_F32>
+template <int NT, int RT, int D, bool CLASS, bool KSCALE, bool OUT_F32>
 __global__ void __launch_bounds__(kDecThreads, 1)
     dbf_decode_stage_kernel(const __grid_constant__ DecodeGroup grp, const int piece) {
   constexpr int NTOK = NT * 8;
   constexpr int NACC = CLASS ? 16 : 4;
-  constexpr int D = kGroupBlocks;
   constexpr int KW = 4 / RT;
   constexpr int ROWS = RT * 16;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -478,9 +479,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
-template <int NT, int RT, bool CLASS, bool KSCALE, bool OUT_F32>
+template <int NT, int RT, int D, bool CLASS, bool KSCALE, bool OUT_F32>
 dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cudaStream_t stream) {
-  auto kernel = dbf_decode_stage_kernel<NT, RT, CLASS, KSCALE, OUT_F32>;
+  auto kernel = dbf_decode_stage_kernel<NT, RT, D, CLASS, KSCALE, OUT_F32>;
   const DecSmem L = dec_smem_layout(piece, batch < NT * 8 ? batch : NT * 8, NT * 8, ks, RT);
   const size_t smem = static_cast<size_t>(L.total);
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -504,19 +505,19 @@ dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cu
   return err == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
-template <int NT, int RT>
+template <int NT, int RT, int D>
 dbf_status launch_rt(const DecodeGroup& g, int batch, bool kscale, bool class_expand, bool out_f32, int ks, int piece,
                      cudaStream_t stream) {
   if (class_expand) {
-    if (kscale) return out_f32 ? launch_typed<NT, RT, true, true, true>(g, batch, ks, piece, stream)
-                               : launch_typed<NT, RT, true, true, false>(g, batch, ks, piece, stream);
-    return out_f32 ? launch_typed<NT, RT, true, false, true>(g, batch, ks, piece, stream)
-                   : launch_typed<NT, RT, true, false, false>(g, batch, ks, piece, stream);
+    if (kscale) return out_f32 ? launch_typed<NT, RT, D, true, true, true>(g, batch, ks, piece, stream)
+                               : launch_typed<NT, RT, D, true, true, false>(g, batch, ks, piece, stream);
+    return out_f32 ? launch_typed<NT, RT, D, true, false, true>(g, batch, ks, piece, stream)
+                   : launch_typed<NT, RT, D, true, false, false>(g, batch, ks, piece, stream);
   }
-  if (kscale) return out_f32 ? launch_typed<NT, RT, false, true, true>(g, batch, ks, piece, stream)
-                             : launch_typed<NT, RT, false, true, false>(g, batch, ks, piece, stream);
-  return out_f32 ? launch_typed<NT, RT, false, false, true>(g, batch, ks, piece, stream)
-                 : launch_typed<NT, RT, false, false, false>(g, batch, ks, piece, stream);
+  if (kscale) return out_f32 ? launch_typed<NT, RT, D, false, true, true>(g, batch, ks, piece, stream)
+                             : launch_typed<NT, RT, D, false, true, false>(g, batch, ks, piece, stream);
+  return out_f32 ? launch_typed<NT, RT, D, false, false, true>(g, batch, ks, piece, stream)
+                 : launch_typed<NT, RT, D, false, false, false>(g, batch, ks, piece, stream);
 }
 
 }  // namespace
@@ -585,8 +586,15 @@ dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_e
     int64_t kc = (grp.layer[g].K + plan.ks - 1) / plan.ks;
     grp.layer[g].kchunk = static_cast<int>((kc + 255) / 256 * 256);
   }
-  if (batch > 8) return launch_rt<2, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
-  return launch_rt<1, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+  int64_t max_blocks = 0;
+  for (int g = 0; g < grp.n; ++g) max_blocks = std::max<int64_t>(max_blocks, grp.layer[g].kchunk / 256);
+  const bool long_rows = max_blocks > 8;
+  if (batch > 8) {
+    return long_rows ? launch_rt<2, 4, 8>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
+                     : launch_rt<2, 4, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+  }
+  return long_rows ? launch_rt<1, 4, 8>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
+                   : launch_rt<1, 4, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
 }
 
 dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
