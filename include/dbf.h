@@ -19,7 +19,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - All data pointers are DEVICE pointers owned by the caller.  The library
- *    never allocates, frees or keeps memory and keeps no state between calls.
+ *    never allocates, frees or keeps memory; apart from cached device properties
+ *    it keeps no state between calls (dbf_forward_noalloc aside, see there).
  *  - fp16 buffers are IEEE binary16 bit patterns (uint16_t), e.g. __half or a
  *    torch.float16 tensor.
  *  - Matrices are row-major and dense (no padding between rows) unless said.
