@@ -123,6 +123,16 @@ __device__ __forceinline__ void st_cluster_v4f32(uint32_t cluster_addr, float a,
                : "memory");
 }
 
+// Asynchronous 16-byte store into another CTA's shared memory of the cluster;
+// its completion is counted in bytes on that CTA's mbarrier (no fence needed).
+__device__ __forceinline__ void st_async_v4f32(uint32_t cluster_addr, float a, float b, float c, float d,
+                                               uint32_t mbar_cluster_addr) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(mbar_cluster_addr)
+               : "memory");
+}
+
 // Bulk copy from this CTA's shared memory into another CTA's shared memory of
 // the cluster; completion is counted in bytes on the destination's mbarrier.
 // Both addresses 16-byte aligned, size a multiple of 16.  (Unicast: one

@@ -323,16 +323,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t local = 0;
     if constexpr (SPLIT) {
       // Reduce-scatter of the ks partial tiles of one (tile, all K) item: rank j
-      // finishes token columns [j*cw, (j+1)*cw).  Each thread (one weight row)
-      // sorts its partial row into the idle A ring by destination rank; after a
-      // cluster barrier (every rank's MMAs are done, so every ring is free) one
-      // thread sends each peer its slice with a bulk copy that completes on the
-      // peer's mbarrier, and each rank adds the ks parts of its own columns in
-      // rank order (deterministic).
+      // finishes token columns [j*cw, (j+1)*cw).  Once every rank's MMAs are
+      // done (a cluster barrier: every operand ring is idle), each thread (one
+      // weight row) reads its partial row out of TMEM and stores each quad of
+      // columns straight into the owning rank's B ring with st.async, counted
+      // in bytes on that rank's mbarrier; its own quads go to its A ring.  All
+      // the CTA's warps then add the ks parts in rank order (deterministic).
       const int cw = NTILE / ks;
       const int cw4 = cw / 4;
       const uint32_t slice_bytes = static_cast<uint32_t>(kBM * cw * 4);
-      float4* part = reinterpret_cast<float4*>(a_st);  // [dst rank][cw4][128 rows]
+      float4* own = reinterpret_cast<float4*>(a_st);   // [cw4][128 rows]
       float4* recv = reinterpret_cast<float4*>(b_st);  // [src rank][cw4][128 rows]
       const int r = q * 32 + lane;
       const int w = blockIdx.x;  // one item per CTA
@@ -341,6 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int b0, b1;
       item_blocks(w, b0, b1);
       const bool have = got && b1 > b0;  // an empty K slice contributes zeros
+      cluster_wait_acquire();    // phase 0: every CTA of the cluster initialised its barriers
+      cluster_arrive_release();  // phase 1: this CTA's MMAs are done, its rings are idle
+      cluster_wait_acquire();
+      if (tid == kWarpEpi0 * 32) mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(ks - 1) * slice_bytes);
       for (int col = 0; col < NTILE; col += 32) {
         uint32_t v[32];
         if (have) {
@@ -353,55 +357,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
           const int c = col + 4 * j4;
-          const int dst = c / cw, cc = c - dst * cw;
-          part[(dst * cw4 + (cc >> 2)) * kBM + r] =
-              make_float4(__uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]), __uint_as_float(v[4 * j4 + 2]),
-                          __uint_as_float(v[4 * j4 + 3]));
-        }
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();  // the partial tile is read by the bulk copies
-      cluster_wait_acquire();    // phase 0: every CTA of the cluster initialised its barriers
-      cluster_arrive_release();  // phase 1: this CTA's MMAs are done and its partial tile is written
-      cluster_wait_acquire();
-      if (tid == kWarpEpi0 * 32) {
-        mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(ks - 1) * slice_bytes);
-        for (int j = 1; j < ks; ++j) {
-          const int dst = (rank + j) % ks;
-          bulk_copy_to_peer(map_to_rank(recv + rank * cw4 * kBM, static_cast<uint32_t>(dst)), part + dst * cw4 * kBM,
-                            slice_bytes, map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
-        }
-      }
-      if (mbar_wait_cluster_bounded(recv_bar, 0, p.status)) {
-        const int m0 = ((w / ks) % m_tiles) * kBM;
-        const int n0 = ((w / ks) / m_tiles) * NTILE + rank * cw;
-        const int row = m0 + r;
-        if (row < p.M) {
-          const float rs = __half2float(p.rowscale[row]);
-          for (int c4 = 0; c4 < cw4; ++c4) {
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int src = 0; src < ks; ++src) {
-              const float4 t = src == rank ? part[(rank * cw4 + c4) * kBM + r] : recv[(src * cw4 + c4) * kBM + r];
-              sum.x += t.x;
-              sum.y += t.y;
-              sum.z += t.z;
-              sum.w += t.w;
-            }
-            const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int tok = n0 + 4 * c4 + e;
-              if (tok < p.batch) {
-                if constexpr (OUT_F32) {
-                  out[static_cast<int64_t>(tok) * p.ld_out + row] = rs * vals[e];
-                } else {
-                  out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(rs * vals[e]);
-                }
-              }
-            }
+          const int dst = c / cw, cc4 = (c - dst * cw) >> 2;
+          const float f0 = __uint_as_float(v[4 * j4]), f1 = __uint_as_float(v[4 * j4 + 1]);
+          const float f2 = __uint_as_float(v[4 * j4 + 2]), f3 = __uint_as_float(v[4 * j4 + 3]);
+          if (dst == rank) {
+            own[cc4 * kBM + r] = make_float4(f0, f1, f2, f3);
+          } else {
+            st_async_v4f32(map_to_rank(&recv[(rank * cw4 + cc4) * kBM + r], static_cast<uint32_t>(dst)), f0, f1, f2,
+                           f3, map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[0]);
     } else {
       constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
       OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
@@ -485,8 +453,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
   if constexpr (SPLIT) {
-    // phase 2: no CTA leaves while a peer's bulk copy may still read from or
-    // write into its shared memory (every rank has waited for its own parts)
+    // split K: every warp adds the ranks' parts of this CTA's token columns
+    // (its own part is in the A ring, the peers' in the B ring) and stores them
+    const int cw = NTILE / ks;
+    const int cw4 = cw / 4;
+    const float4* own = reinterpret_cast<const float4*>(a_st);
+    const float4* recv = reinterpret_cast<const float4*>(b_st);
+    const int w = blockIdx.x;
+    if (mbar_wait_cluster_bounded(recv_bar, 0, p.status)) {
+      using OutT = typename std::conditional<OUT_F32, float, __half>::type;
+      OutT* out = static_cast<OutT*>(p.out);
+      const int m0 = ((w / ks) % m_tiles) * kBM;
+      const int n0 = ((w / ks) / m_tiles) * NTILE + rank * cw;
+      for (int idx = tid; idx < kBM * cw4; idx += kThreads) {
+        const int r = idx & (kBM - 1), c4 = idx >> 7;  // consecutive threads: consecutive rows
+        const int row = m0 + r;
+        if (row >= p.M) continue;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < ks; ++src) {
+          const float4 t = src == rank ? own[c4 * kBM + r] : recv[(src * cw4 + c4) * kBM + r];
+          sum.x += t.x;
+          sum.y += t.y;
+          sum.z += t.z;
+          sum.w += t.w;
+        }
+        const float rs = __half2float(p.rowscale[row]);
+        const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = n0 + 4 * c4 + e;
+          if (tok < p.batch) {
+            if constexpr (OUT_F32) {
+              out[static_cast<int64_t>(tok) * p.ld_out + row] = rs * vals[e];
+            } else {
+              out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(rs * vals[e]);
+            }
+          }
+        }
+      }
+    }
+    // phase 2: no CTA leaves while a peer may still store into its shared
+    // memory (every rank has waited for all of its parts)
     cluster_arrive_release();
     cluster_wait_acquire();
   }
