@@ -118,7 +118,7 @@ __host__ __device__ inline DecSmem dec_smem_layout(int piece, int nvalid, int nt
 // KW = 4/RT K slices; a cluster of ks CTAs along K splits the reduction further.
 // The launch may cover several layers that share their input (a group): the
 // CTA's tile index picks its layer.
-template <int NT, int RT, int D, bool CLASS, bool KSCALE, bool OUT_F32>
+template <int NT, int RT, int D, bool TOKPAR, bool CLASS, bool KSCALE, bool OUT_F32>
 __global__ void __launch_bounds__(kDecThreads, 1)
     dbf_decode_stage_kernel(const __grid_constant__ DecodeGroup grp, const int piece) {
   constexpr int NTOK = NT * 8;
@@ -261,10 +261,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     // ---- u = fp16(x (.) b) in place; class sums U_rest (all groups but 15),
     // per-warp parts added in warp order (deterministic).
-    // Up to 8 tokens: all 128 threads take each token's row in turn.
-    // 9 to 16 tokens: warp w owns tokens w, w+4, w+8, w+12; a thread scales and
+    // Up to 3 tokens: all 128 threads take each token's row in turn.
+    // 4 to 16 tokens: warp w owns tokens w, w+4, w+8, w+12; a thread scales and
     // sums only what it owns, so a warp's tokens run side by side.
-    if constexpr (NT == 1) {
+    if constexpr (!TOKPAR) {
       if constexpr (KSCALE || CLASS) {
         const int nch = plen / 8;
         for (int tok = 0; tok < nvalid; ++tok) {
@@ -479,9 +479,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
-template <int NT, int RT, int D, bool CLASS, bool KSCALE, bool OUT_F32>
+template <int NT, int RT, int D, bool TOKPAR, bool CLASS, bool KSCALE, bool OUT_F32>
 dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cudaStream_t stream) {
-  auto kernel = dbf_decode_stage_kernel<NT, RT, D, CLASS, KSCALE, OUT_F32>;
+  auto kernel = dbf_decode_stage_kernel<NT, RT, D, TOKPAR, CLASS, KSCALE, OUT_F32>;
   const DecSmem L = dec_smem_layout(piece, batch < NT * 8 ? batch : NT * 8, NT * 8, ks, RT);
   const size_t smem = static_cast<size_t>(L.total);
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -505,19 +505,19 @@ dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cu
   return err == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
-template <int NT, int RT, int D>
+template <int NT, int RT, int D, bool TOKPAR>
 dbf_status launch_rt(const DecodeGroup& g, int batch, bool kscale, bool class_expand, bool out_f32, int ks, int piece,
                      cudaStream_t stream) {
   if (class_expand) {
-    if (kscale) return out_f32 ? launch_typed<NT, RT, D, true, true, true>(g, batch, ks, piece, stream)
-                               : launch_typed<NT, RT, D, true, true, false>(g, batch, ks, piece, stream);
-    return out_f32 ? launch_typed<NT, RT, D, true, false, true>(g, batch, ks, piece, stream)
-                   : launch_typed<NT, RT, D, true, false, false>(g, batch, ks, piece, stream);
+    if (kscale) return out_f32 ? launch_typed<NT, RT, D, TOKPAR, true, true, true>(g, batch, ks, piece, stream)
+                               : launch_typed<NT, RT, D, TOKPAR, true, true, false>(g, batch, ks, piece, stream);
+    return out_f32 ? launch_typed<NT, RT, D, TOKPAR, true, false, true>(g, batch, ks, piece, stream)
+                   : launch_typed<NT, RT, D, TOKPAR, true, false, false>(g, batch, ks, piece, stream);
   }
-  if (kscale) return out_f32 ? launch_typed<NT, RT, D, false, true, true>(g, batch, ks, piece, stream)
-                             : launch_typed<NT, RT, D, false, true, false>(g, batch, ks, piece, stream);
-  return out_f32 ? launch_typed<NT, RT, D, false, false, true>(g, batch, ks, piece, stream)
-                 : launch_typed<NT, RT, D, false, false, false>(g, batch, ks, piece, stream);
+  if (kscale) return out_f32 ? launch_typed<NT, RT, D, TOKPAR, false, true, true>(g, batch, ks, piece, stream)
+                             : launch_typed<NT, RT, D, TOKPAR, false, true, false>(g, batch, ks, piece, stream);
+  return out_f32 ? launch_typed<NT, RT, D, TOKPAR, false, false, true>(g, batch, ks, piece, stream)
+                 : launch_typed<NT, RT, D, TOKPAR, false, false, false>(g, batch, ks, piece, stream);
 }
 
 }  // namespace
@@ -589,12 +589,17 @@ dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_e
   int64_t max_blocks = 0;
   for (int g = 0; g < grp.n; ++g) max_blocks = std::max<int64_t>(max_blocks, grp.layer[g].kchunk / 256);
   const bool long_rows = max_blocks > 8;
+  // the activation pass: row by row for 1-3 tokens, four tokens per warp side by side from 4
   if (batch > 8) {
-    return long_rows ? launch_rt<2, 4, 8>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
-                     : launch_rt<2, 4, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+    return long_rows ? launch_rt<2, 4, 8, true>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
+                     : launch_rt<2, 4, 4, true>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
   }
-  return long_rows ? launch_rt<1, 4, 8>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
-                   : launch_rt<1, 4, 4>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+  if (batch >= 4) {
+    return long_rows ? launch_rt<1, 4, 8, true>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
+                     : launch_rt<1, 4, 4, true>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
+  }
+  return long_rows ? launch_rt<1, 4, 8, false>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
+                   : launch_rt<1, 4, 4, false>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
 }
 
 dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
