@@ -52,8 +52,9 @@ namespace {
 
 constexpr int kDecThreads = 128;
 // 256-column blocks per register group of weights: 4, or 8 for rows of more
-// than 8 blocks per warp (long reductions stream their weights; a bigger group
-// keeps more of them in flight while the previous group is multiplied)
+// than 8 blocks per warp in launches of at most 1.75 CTAs per SM (long
+// reductions stream their weights; a bigger group keeps more of them in flight
+// while the previous group is multiplied)
 constexpr int kMaxClusterK = 8;
 constexpr int kSmemBudget = 100 * 1024;
 constexpr int kHeadBytes = 512;  // mbarriers, abort flag, class sums and their per-warp parts
@@ -588,7 +589,9 @@ dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_e
   }
   int64_t max_blocks = 0;
   for (int g = 0; g < grp.n; ++g) max_blocks = std::max<int64_t>(max_blocks, grp.layer[g].kchunk / 256);
-  const bool long_rows = max_blocks > 8;
+  // 8-block groups cost registers: keep them to launches of at most 1.75 CTAs
+  // per SM, where the neighbouring launch is not resident beside them anyway
+  const bool long_rows = max_blocks > 8 && 4 * tiles * plan.ks <= 7 * static_cast<int64_t>(dev.num_sms);
   // the activation pass: row by row for 1-3 tokens, four tokens per warp side by side from 4
   if (batch > 8) {
     return long_rows ? launch_rt<2, 4, 8, true>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream)
