@@ -32,12 +32,12 @@
 //               in shared memory -> 16-byte global stores (warp w reads TMEM
 //               lanes 32*(w%4) .. 32*(w%4)+31).
 // Few tiles (small batches): the K range of each 128 x 128 tile is split over a
-// cluster of 2-8 CTAs, one (tile, K slice) per CTA.  After the main loop each
-// CTA sorts its fp32 partial tile by destination rank into its idle A ring; a
-// cluster barrier says every ring is idle; one thread bulk-copies each peer its
-// slice into the peer's B ring (completion counted on the peer's mbarrier), and
-// every rank finishes its share of the token columns, adding the parts in rank
-// order.
+// cluster of 2-8 CTAs, one (tile, K slice) per CTA.  After the main loop a
+// cluster barrier says every CTA's operand rings are idle; all warps then read
+// the fp32 partial tile out of TMEM and store each rank's share of the token
+// columns straight into that rank's B ring (st.async, completion counted in
+// bytes on the rank's mbarrier), and every rank finishes its share, adding the
+// parts in rank order.
 // Stage hand-off is through mbarriers; every wait is bounded and an expired
 // wait records DBF_ERR_TIMEOUT in the workspace status word, raises a CTA-wide
 // abort flag and lets all roles fall through to the teardown, which frees TMEM
@@ -75,7 +75,9 @@ struct Cfg {
   static constexpr int kBarOffset = kEpiOffset + 4 * kEpiStageBytes;
   // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done, recv
   static constexpr int kNumBars = 3 * kStages + 6;
-  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;  // + tmem slot/abort + align slack
+  static constexpr int kRsOffset = kBarOffset + kNumBars * 8 + 16;  // after the tmem slot and abort flag
+  // + split K: the tile's row scales (fp32), + alignment slack
+  static constexpr int kSmemBytes = kRsOffset + kBM * 4 + 1024;
   static constexpr int kTmemCols = 2 * NTILE;
   // split K: once a CTA's MMAs are done its operand ring is idle; the A ring
   // then holds this CTA's fp32 partial tile sorted by destination rank and the
@@ -105,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* recv_bar = bars + 3 * S + 5;  // split K: the peers' parts have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* rs_s = reinterpret_cast<float*>(smem + C::kRsOffset);  // split K: row scales of the tile
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -322,67 +325,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     OutT* out = static_cast<OutT*>(p.out);
     uint32_t local = 0;
     if constexpr (SPLIT) {
-      // Reduce-scatter of the ks partial tiles of one (tile, all K) item: rank j
-      // finishes token columns [j*cw, (j+1)*cw).  Once every rank's MMAs are
-      // done (a cluster barrier: every operand ring is idle), each thread (one
-      // weight row) reads its partial row out of TMEM and stores each quad of
-      // columns straight into the owning rank's B ring with st.async, counted
-      // in bytes on that rank's mbarrier; its own quads go to its A ring.  All
-      // the CTA's warps then add the ks parts in rank order (deterministic).
-      const int cw = NTILE / ks;
-      const int cw4 = cw / 4;
-      const uint32_t slice_bytes = static_cast<uint32_t>(kBM * cw * 4);
-      float4* own = reinterpret_cast<float4*>(a_st);   // [cw4][128 rows]
-      float4* recv = reinterpret_cast<float4*>(b_st);  // [src rank][cw4][128 rows]
+      // split K: the exchange and the reduction run on all warps after the
+      // role loops; the epilogue warps only stage the tile's row scales here
+      if (!p.weights_early) pdl_wait();
       const int r = q * 32 + lane;
-      const int w = blockIdx.x;  // one item per CTA
-      const bool got = mbar_wait_bounded(&acc_full[0], 0, abort_flag, p.status);
-      tc_fence_after();
-      int b0, b1;
-      item_blocks(w, b0, b1);
-      const bool have = got && b1 > b0;  // an empty K slice contributes zeros
-      cluster_wait_acquire();    // phase 0: every CTA of the cluster initialised its barriers
-      cluster_arrive_release();  // phase 1: this CTA's MMAs are done, its rings are idle
-      cluster_wait_acquire();
-      if (tid == kWarpEpi0 * 32) mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(ks - 1) * slice_bytes);
-      for (int col = 0; col < NTILE; col += 32) {
-        uint32_t v[32];
-        if (have) {
-          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col), v);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0u;
-        }
-#pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-          const int c = col + 4 * j4;
-          const int dst = c / cw, cc4 = (c - dst * cw) >> 2;
-          const float f0 = __uint_as_float(v[4 * j4]), f1 = __uint_as_float(v[4 * j4 + 1]);
-          const float f2 = __uint_as_float(v[4 * j4 + 2]), f3 = __uint_as_float(v[4 * j4 + 3]);
-          if (dst == rank) {
-            own[cc4 * kBM + r] = make_float4(f0, f1, f2, f3);
-          } else {
-            st_async_v4f32(map_to_rank(&recv[(rank * cw4 + cc4) * kBM + r], static_cast<uint32_t>(dst)), f0, f1, f2,
-                           f3, map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[0]);
+      const int row = ((static_cast<int>(blockIdx.x) / ks) % m_tiles) * kBM + r;
+      rs_s[r] = row < p.M ? __half2float(p.rowscale[row]) : 0.f;
     } else {
       constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
       OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
       const bool ld_ok = (p.ld_out % kVec) == 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
         const uint32_t buf = local & 1;
-        if (!mbar_wait_bounded(&acc_full[buf], (local >> 1) & 1, abort_flag, p.status)) break;
-        tc_fence_after();
         const int m0 = (tile % m_tiles) * kBM;
         const int n0 = (tile / m_tiles) * NTILE;
         const int row0 = m0 + q * 32;
         const int row = row0 + lane;
-        const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;
+        const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;  // in flight during the wait
+        if (!mbar_wait_bounded(&acc_full[buf], (local >> 1) & 1, abort_flag, p.status)) break;
+        tc_fence_after();
         const bool rows_full = row0 + 32 <= p.M;
         for (int col = 0; col < NTILE; col += 32) {
           if (n0 + col >= p.batch) break;  // warp-uniform
@@ -433,15 +394,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ------------------------------------------------ teardown
+  // ------------------------------------------------ split K: exchange of the partial tiles
   if constexpr (SPLIT) {
-    if (warp < kWarpEpi0) {  // the epilogue warps passed phases 0 and 1 above
-      __syncwarp();
-      cluster_wait_acquire();
-      cluster_arrive_release();
-      cluster_wait_acquire();
+    // Reduce-scatter of the ks partial tiles of one (tile, all K) item: rank j
+    // finishes token columns [j*cw, (j+1)*cw).  Once every rank's MMAs are done
+    // (a cluster barrier: every operand ring is idle), all 14 warps read the
+    // partial tile out of TMEM (warp w may read lanes 32*(w%4) .. 32*(w%4)+31;
+    // the warps of a lane quadrant share its 16-column chunks) and store each
+    // quad of columns straight into the owning rank's B ring with st.async,
+    // counted in bytes on that rank's mbarrier; the quads this rank owns go to
+    // its A ring.
+    __syncwarp();  // the single-thread roles rejoin their warps
+    constexpr int kWarps = kThreads / 32;
+    const int cw = NTILE / ks;
+    const int cw4 = cw / 4;
+    const uint32_t slice_bytes = static_cast<uint32_t>(kBM * cw * 4);
+    float4* own = reinterpret_cast<float4*>(a_st);   // [cw4][128 rows]
+    float4* recv = reinterpret_cast<float4*>(b_st);  // [src rank][cw4][128 rows]
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const bool got = mbar_wait_bounded(&acc_full[0], 0, abort_flag, p.status);
+    tc_fence_after();
+    int b0, b1;
+    item_blocks(blockIdx.x, b0, b1);
+    const bool have = __all_sync(0xffffffffu, got) && b1 > b0;  // an empty K slice contributes zeros
+    cluster_wait_acquire();    // phase 0: every CTA of the cluster initialised its barriers
+    cluster_arrive_release();  // phase 1: this CTA's MMAs are done, its rings are idle
+    cluster_wait_acquire();
+    if (tid == 0) mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(ks - 1) * slice_bytes);
+    const int nq = (kWarps - q + 3) / 4;  // warps that may read quadrant q (4, 4, 3, 3)
+    for (int col = 16 * (warp >> 2); col < NTILE; col += 16 * nq) {
+      uint32_t v[16];
+      if (have) {
+        tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col), v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0u;
+      }
+#pragma unroll
+      for (int j4 = 0; j4 < 4; ++j4) {
+        const int c = col + 4 * j4;
+        const int dst = c / cw, cc4 = (c - dst * cw) >> 2;
+        const float f0 = __uint_as_float(v[4 * j4]), f1 = __uint_as_float(v[4 * j4 + 1]);
+        const float f2 = __uint_as_float(v[4 * j4 + 2]), f3 = __uint_as_float(v[4 * j4 + 3]);
+        if (dst == rank) {
+          own[cc4 * kBM + r] = make_float4(f0, f1, f2, f3);
+        } else {
+          st_async_v4f32(map_to_rank(&recv[(rank * cw4 + cc4) * kBM + r], static_cast<uint32_t>(dst)), f0, f1, f2, f3,
+                         map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
+        }
+      }
     }
   }
+
+  // ------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
@@ -477,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sum.z += t.z;
           sum.w += t.w;
         }
-        const float rs = __half2float(p.rowscale[row]);
+        const float rs = rs_s[r];
         const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
