@@ -79,12 +79,12 @@ struct Cfg {
   // + split K: the tile's row scales (fp32), + alignment slack
   static constexpr int kSmemBytes = kRsOffset + kBM * 4 + 1024;
   static constexpr int kTmemCols = 2 * NTILE;
-  // split K: once a CTA's MMAs are done its operand ring is idle; the A ring
-  // then holds this CTA's fp32 partial tile sorted by destination rank and the
-  // B ring receives the peers' parts, both [rank][NTILE/ks/4][128 rows] float4.
+  // split K: once a CTA's MMAs are done its operand rings are idle; the B ring
+  // then receives the peers' parts of this CTA's token columns,
+  // [src rank][NTILE/ks/4][128 rows] float4 (at most one whole partial tile).
   static constexpr int kPartialBytes = kBM * NTILE * 4;
-  static_assert(!SPLIT || (kPartialBytes <= kStages * kABytes && kPartialBytes <= kStages * kBBytes),
-                "split-K partial tiles must fit in the idle operand ring");
+  static_assert(!SPLIT || kPartialBytes <= kStages * kBBytes, "split-K parts must fit in the idle B ring");
+  static_assert(!SPLIT || 14 * 8 * 32 * 4 <= 4 * kEpiStageBytes, "split-K output transposes must fit the epilogue stage");
 };
 
 template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32>
@@ -401,18 +401,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (a cluster barrier: every operand ring is idle), all 14 warps read the
     // partial tile out of TMEM (warp w may read lanes 32*(w%4) .. 32*(w%4)+31;
     // the warps of a lane quadrant share its 16-column chunks) and store each
-    // quad of columns straight into the owning rank's B ring with st.async,
-    // counted in bytes on that rank's mbarrier; the quads this rank owns go to
-    // its A ring.
+    // quad of the other ranks' columns straight into the owning rank's B ring
+    // with st.async, counted in bytes on that rank's mbarrier.  This rank's own
+    // columns stay in TMEM.
     __syncwarp();  // the single-thread roles rejoin their warps
     constexpr int kWarps = kThreads / 32;
     const int cw = NTILE / ks;
     const int cw4 = cw / 4;
     const uint32_t slice_bytes = static_cast<uint32_t>(kBM * cw * 4);
-    float4* own = reinterpret_cast<float4*>(a_st);   // [cw4][128 rows]
     float4* recv = reinterpret_cast<float4*>(b_st);  // [src rank][cw4][128 rows]
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    const int nq = (kWarps - q + 3) / 4;  // warps that may read quadrant q (4, 4, 3, 3)
+    const int jq = warp >> 2;             // this warp's index among them
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const bool got = mbar_wait_bounded(&acc_full[0], 0, abort_flag, p.status);
     tc_fence_after();
     int b0, b1;
@@ -422,27 +424,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_arrive_release();  // phase 1: this CTA's MMAs are done, its rings are idle
     cluster_wait_acquire();
     if (tid == 0) mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(ks - 1) * slice_bytes);
-    const int nq = (kWarps - q + 3) / 4;  // warps that may read quadrant q (4, 4, 3, 3)
-    for (int col = 16 * (warp >> 2); col < NTILE; col += 16 * nq) {
+    for (int col = 16 * jq; col < NTILE; col += 16 * nq) {
+      const int dst = col / cw;  // cw >= 16: a chunk has one owner
+      if (dst == rank) continue;
       uint32_t v[16];
       if (have) {
-        tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(col), v);
+        tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(col), v);
         tmem_ld_wait();
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0u;
       }
+      const int cc40 = (col - dst * cw) >> 2;
 #pragma unroll
       for (int j4 = 0; j4 < 4; ++j4) {
-        const int c = col + 4 * j4;
-        const int dst = c / cw, cc4 = (c - dst * cw) >> 2;
-        const float f0 = __uint_as_float(v[4 * j4]), f1 = __uint_as_float(v[4 * j4 + 1]);
-        const float f2 = __uint_as_float(v[4 * j4 + 2]), f3 = __uint_as_float(v[4 * j4 + 3]);
-        if (dst == rank) {
-          own[cc4 * kBM + r] = make_float4(f0, f1, f2, f3);
+        st_async_v4f32(map_to_rank(&recv[(rank * cw4 + cc40 + j4) * kBM + r], static_cast<uint32_t>(dst)),
+                       __uint_as_float(v[4 * j4]), __uint_as_float(v[4 * j4 + 1]), __uint_as_float(v[4 * j4 + 2]),
+                       __uint_as_float(v[4 * j4 + 3]), map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
+      }
+    }
+
+    // Finish this rank's columns once the peers' parts have landed: thread r of
+    // quadrant q adds, for its row and 8 of the columns, the ks parts in rank
+    // order (its own from TMEM), scales, and the warp writes its 32 rows x 8
+    // tokens through a shared-memory transpose with 16-byte stores.
+    const bool rcv = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(recv_bar, 0, p.status));
+    if (rcv) {
+      using OutT = typename std::conditional<OUT_F32, float, __half>::type;
+      constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
+      OutT* out = static_cast<OutT*>(p.out);
+      OutT* stg = reinterpret_cast<OutT*>(epi_st + warp * (8 * 32 * sizeof(OutT)));  // [8 tokens][32 rows]
+      const int m0 = ((static_cast<int>(blockIdx.x) / ks) % m_tiles) * kBM;
+      const int n0 = ((static_cast<int>(blockIdx.x) / ks) / m_tiles) * NTILE + rank * cw;
+      const int row0 = m0 + q * 32;
+      const int row = row0 + lane;
+      const float rs = rs_s[r];
+      const bool vec_ok = row0 + 32 <= p.M && (p.ld_out % kVec) == 0;
+      for (int ch = jq; ch < cw / 8; ch += nq) {
+        uint32_t v[8];
+        if (have) {
+          tmem_ld_32x32b_x8(lane_base + static_cast<uint32_t>(rank * cw + 8 * ch), v);
+          tmem_ld_wait();
         } else {
-          st_async_v4f32(map_to_rank(&recv[(rank * cw4 + cc4) * kBM + r], static_cast<uint32_t>(dst)), f0, f1, f2, f3,
-                         map_to_rank(recv_bar, static_cast<uint32_t>(dst)));
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = 0u;
+        }
+        float sum[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum[j] = 0.f;
+        for (int src = 0; src < ks; ++src) {
+          float t[8];
+          if (src == rank) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t[j] = __uint_as_float(v[j]);
+          } else {
+            const float4 lo = recv[(src * cw4 + 2 * ch) * kBM + r];
+            const float4 hi = recv[(src * cw4 + 2 * ch + 1) * kBM + r];
+            t[0] = lo.x; t[1] = lo.y; t[2] = lo.z; t[3] = lo.w;
+            t[4] = hi.x; t[5] = hi.y; t[6] = hi.z; t[7] = hi.w;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sum[j] += t[j];
+        }
+        const int tok0 = n0 + 8 * ch;
+        if (vec_ok && tok0 + 8 <= p.batch) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if constexpr (OUT_F32) {
+              stg[j * 32 + lane] = rs * sum[j];
+            } else {
+              stg[j * 32 + lane] = __float2half_rn(rs * sum[j]);
+            }
+          }
+          __syncwarp();
+          constexpr int kChunksPerTok = 32 / kVec;
+#pragma unroll
+          for (int m = 0; m < 8 * kChunksPerTok / 32; ++m) {
+            const int cidx = lane + 32 * m;
+            const int tk = cidx / kChunksPerTok, rp = cidx % kChunksPerTok;
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + tk * 32 + rp * kVec);
+            *reinterpret_cast<uint4*>(out + static_cast<int64_t>(tok0 + tk) * p.ld_out + row0 + rp * kVec) = val;
+          }
+          __syncwarp();
+        } else if (row < p.M) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int tok = tok0 + j;
+            if (tok < p.batch) {
+              if constexpr (OUT_F32) {
+                out[static_cast<int64_t>(tok) * p.ld_out + row] = rs * sum[j];
+              } else {
+                out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(rs * sum[j]);
+              }
+            }
+          }
         }
       }
     }
@@ -460,45 +535,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
   if constexpr (SPLIT) {
-    // split K: every warp adds the ranks' parts of this CTA's token columns
-    // (its own part is in the A ring, the peers' in the B ring) and stores them
-    const int cw = NTILE / ks;
-    const int cw4 = cw / 4;
-    const float4* own = reinterpret_cast<const float4*>(a_st);
-    const float4* recv = reinterpret_cast<const float4*>(b_st);
-    const int w = blockIdx.x;
-    if (mbar_wait_cluster_bounded(recv_bar, 0, p.status)) {
-      using OutT = typename std::conditional<OUT_F32, float, __half>::type;
-      OutT* out = static_cast<OutT*>(p.out);
-      const int m0 = ((w / ks) % m_tiles) * kBM;
-      const int n0 = ((w / ks) / m_tiles) * NTILE + rank * cw;
-      for (int idx = tid; idx < kBM * cw4; idx += kThreads) {
-        const int r = idx & (kBM - 1), c4 = idx >> 7;  // consecutive threads: consecutive rows
-        const int row = m0 + r;
-        if (row >= p.M) continue;
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < ks; ++src) {
-          const float4 t = src == rank ? own[c4 * kBM + r] : recv[(src * cw4 + c4) * kBM + r];
-          sum.x += t.x;
-          sum.y += t.y;
-          sum.z += t.z;
-          sum.w += t.w;
-        }
-        const float rs = rs_s[r];
-        const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int tok = n0 + 4 * c4 + e;
-          if (tok < p.batch) {
-            if constexpr (OUT_F32) {
-              out[static_cast<int64_t>(tok) * p.ld_out + row] = rs * vals[e];
-            } else {
-              out[static_cast<int64_t>(tok) * p.ld_out + row] = __float2half_rn(rs * vals[e]);
-            }
-          }
-        }
-      }
-    }
     // phase 2: no CTA leaves while a peer may still store into its shared
     // memory (every rank has waited for all of its parts)
     cluster_arrive_release();
