@@ -661,6 +661,33 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
   if (static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + ntile - 1) / ntile) * ks > 0x7fffffffLL)
     return DBF_ERR_UNSUPPORTED_SHAPE;
 
+  // Wave tail.  Without a split the persistent CTAs walk the tiles in waves of
+  // one tile per SM, and a last, nearly empty wave costs a whole tile time (896
+  // tiles on 148 SMs: 7 rounds for 6.05 tiles' worth of work).  When leaving
+  // out the last few row tiles (at most a quarter of the SMs' worth of tiles)
+  // makes the rest whole waves, those rows go to a second launch of their own,
+  // which the planner above gives a K split over clusters.
+  if (ks == 1) {
+    const int64_t m_tiles = (a.M + kBM - 1) / kBM;
+    const int64_t n_tiles = (a.batch + ntile - 1) / ntile;
+    if (m_tiles * n_tiles > dev.num_sms && (m_tiles * n_tiles) % dev.num_sms != 0) {
+      for (int64_t t = 1; t < m_tiles && 4 * t * n_tiles <= dev.num_sms; ++t) {
+        if ((m_tiles - t) * n_tiles % dev.num_sms != 0) continue;
+        const int64_t rows_main = (m_tiles - t) * kBM;
+        PrefillArgs head = a;
+        head.M = static_cast<int>(rows_main);
+        PrefillArgs tail = a;
+        tail.M = a.M - static_cast<int>(rows_main);
+        tail.packed = a.packed + rows_main * a.wpr;
+        tail.rowscale = a.rowscale + rows_main;
+        tail.out = static_cast<char*>(a.out) + rows_main * (out_f32 ? 4 : 2);
+        const dbf_status st = launch_prefill_gemm(head, act, act_rows, out_f32, dev, stream);
+        if (st != DBF_OK) return st;
+        return launch_prefill_gemm(tail, act, act_rows, out_f32, dev, stream);
+      }
+    }
+  }
+
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(act_rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};

@@ -184,6 +184,40 @@ def test_ragged_fp16(dbf, path, n, k, m_in, batch):
     assert_fp16_close(y, L.oracle(), f"{path} {n}x{k}x{m_in} b{batch}")
 
 
+# ------------------------------------------------------------------ wave tail of the persistent GEMM
+def _tail_rows(batch):
+    """Output rows n for which the second product's persistent launch (128-row x
+    256-token tiles, one tile per SM per wave) would end in a wave of n_tiles
+    tiles: the last 128-row tile (ragged: 91 rows) then goes to a split-K launch
+    of its own."""
+    from math import gcd
+
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n_tiles = (batch + 255) // 256
+    m_tiles = sms // gcd(n_tiles, sms) + 1
+    return m_tiles * 128 - 37
+
+
+@pytest.mark.parametrize("batch", [256, 2048])
+def test_wave_tail_int_bit_exact(dbf, batch):
+    n, k, m_in = _tail_rows(batch), 1024, 256  # K = 1024: the tail launch splits K 4 ways
+    rng = np.random.default_rng(n + batch)
+    A, B = gen.sign_matrix(rng, n, k), gen.sign_matrix(rng, k, m_in)
+    x = gen.integer_activations(rng, batch, m_in, -8, 8)
+    ones = np.ones
+    L = Layer(dbf, A, B, ones(n, np.float16), ones(k, np.float16), ones(m_in, np.float16), x)
+    y = L.forward(flags=PATHS["prefill"], y_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    assert np.array_equal(y, L.oracle())
+
+
+@pytest.mark.parametrize("batch", [256, 2048])
+def test_wave_tail_fp16(dbf, batch):
+    n = _tail_rows(batch)
+    L = random_layer(dbf, n, 1024, 256, batch, seed=n + batch + 1, scales="lognormal")
+    y = L.forward(flags=PATHS["prefill"]).float().cpu().numpy()
+    assert_fp16_close(y, L.oracle(), f"wave tail {n}x1024x256 b{batch}")
+
+
 def test_fp32_output_matches_fp16_output(dbf):
     L = random_layer(dbf, 256, 128, 256, 4, seed=3)
     for flags in PATHS.values():
