@@ -64,10 +64,17 @@ def layer_flops(n, k, m_in, batch):
     return 2.0 * batch * k * (m_in + n)
 
 
-def kernel_source_hash():
+# Sources each path's kernels and their launches are built from (the others
+# do not change what that path runs).
+DECODE_SOURCES = ("dbf_api.cu", "dbf_device.cuh", "dbf_internal.h", "decode.cu")
+PREFILL_SOURCES = ("dbf_api.cu", "dbf_device.cuh", "dbf_internal.h", "prefill.cu")
+
+
+def kernel_source_hash(files=None):
+    """Hash of the kernel sources (all of csrc, or the named files of it)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "binary_factorized_weight_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -80,7 +87,7 @@ def traffic_for(workload_key):
         with open(path) as f:
             t = json.load(f)
         entry = t[workload_key]
-        if entry.get("source_hash") != kernel_source_hash():
+        if entry.get("source_hash") != kernel_source_hash(entry.get("source_files")):
             return None
         return entry["dram_bytes_per_forward"]
     except Exception:
