@@ -80,6 +80,30 @@ def kernel_source_hash(files=None):
     return h.hexdigest()[:16]
 
 
+def graph_kernel_launches(graph):
+    """Kernel nodes of a captured CUDA graph: the launches one replay makes
+    (None when the graph cannot be inspected)."""
+    try:
+        from cuda.bindings import runtime as rt
+
+        handle = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, count = rt.cudaGraphGetNodes(handle, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, count = rt.cudaGraphGetNodes(handle, count)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kernels = 0
+        for node in nodes[:count]:
+            err, kind = rt.cudaGraphNodeGetType(node)
+            if err != rt.cudaError_t.cudaSuccess:
+                return None
+            kernels += kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        return kernels
+    except Exception:
+        return None
+
+
 def traffic_for(workload_key):
     """DRAM bytes per forward from the committed ncu summary, if the kernels are unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -274,9 +298,10 @@ class Workload:
             self.forward_all()
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)  # kept so that its launches can be counted
         with torch.cuda.graph(g):
             self.forward_all()
+        g.instantiate()
         torch.cuda.synchronize()
         return g
 
@@ -363,6 +388,13 @@ def run_ours(args, shape, batch):
     peaks = load_peaks()
     wl = Workload(dbf, torch, shape, batch, device)
     graph = wl.capture()
+    # launches per step, counted in the captured graph (the planner may split a
+    # product into more than one launch); the per-path formula if it cannot be read
+    step_launches = graph_kernel_launches(graph)
+    launches_source = "counted in the captured graph"
+    if step_launches is None:
+        step_launches = wl.copies * wl.launches_per_forward
+        launches_source = "per-path formula"
 
     def barrier():
         if world > 1:
@@ -494,7 +526,8 @@ def run_ours(args, shape, batch):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 2)},
-        "gpu_launches": args.steps * wl.copies * wl.launches_per_forward,
+        "gpu_launches": args.steps * step_launches,
+        "gpu_launches_source": launches_source,
         "clocks": clocks,
     }
     if batch > 16:
