@@ -149,7 +149,9 @@ DBF_API size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, i
  * the sign operand exactly.  With a = m = b = 1, integer x and |t| <= 2048,
  * every step is exact and fp32 output equals the integer result.
  * Paths: batch <= 16 runs two PDL-chained sign-GEMV kernels (mma.sync);
- * larger batches run two tcgen05 tensor-core kernels.
+ * larger batches run the two products as tcgen05 tensor-core GEMMs, one
+ * launch each, or two when a GEMM's last wave of tiles would leave most SMs
+ * idle (its last rows then run as a split-K launch of their own).
  * Shape contract: n >= 1, batch >= 1, k and m_in multiples of 64 in
  * [64, 1 << 20], n and batch <= 1 << 24.  All pointers 16-byte aligned;
  * outputs must not overlap inputs.
