@@ -27,6 +27,8 @@ def _setup(lib):
     """Declare the C signatures on a loaded oracle library."""
     i64, dbl, vp = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
     lib.oracle_words_per_row.argtypes = [i64]
     lib.oracle_words_per_row.restype = i64
     lib.oracle_unpack_signs.argtypes = [vp, i64, i64, vp]
@@ -39,6 +41,8 @@ def _setup(lib):
     lib.oracle_forward_transposed.restype = None
     lib.oracle_dense_weight.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
     lib.oracle_dense_weight.restype = None
+    lib.oracle_bqq_dense_weight.argtypes = [vp, vp, vp, vp, vp, dbl, i64, i64, i64, i64, vp]
+    lib.oracle_bqq_dense_weight.restype = None
     lib.oracle_forward_dense.argtypes = [vp, vp, i64, i64, i64, vp]
     lib.oracle_forward_dense.restype = None
     lib.oracle_bits_per_weight.argtypes = [i64, i64, i64]
@@ -86,8 +90,13 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's loops use (timing only; the results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))
+
+
 def words_per_row(cols: int) -> int:
-    """32-bit words per packed row (rows are padded to 128 bits)."""
+    """32-bit words per packed row (rows are padded to whole 256-column blocks of 8 words)."""
     return int(_load().oracle_words_per_row(cols))
 
 
@@ -192,3 +201,27 @@ def bits_per_weight(n: int, k: int, m_in: int) -> float:
 def scale_bits_per_weight(n: int, k: int, m_in: int) -> float:
     """fp16 scale-vector bits per dense weight, 16(n + k + m_in)/(n m_in)."""
     return float(_load().oracle_scale_bits_per_weight(n, k, m_in))
+
+
+def bqq_dense_weight(Y, Z, r, s, t, u) -> np.ndarray:
+    """W = sum_i (r_i Y_i Z_i + s_i Y_i 1_Z + t_i 1_Y Z_i) + u 1 (sciencestack.ai page of "Binary Quadratic
+    Quantization", TL;DR formula), fp64.  Y: p x n x k and Z: p x k x m binary {0, 1}; r, s, t: p; u scalar."""
+    lib = _load()
+    Y, Z = _i8(Y), _i8(Z)
+    if Y.ndim == 2:
+        Y, Z = Y[None], Z[None]
+    p, n, k = Y.shape
+    p2, k2, m = Z.shape
+    r, s, t = _f64(r).reshape(-1), _f64(s).reshape(-1), _f64(t).reshape(-1)
+    if p2 != p or k2 != k or r.size != p or s.size != p or t.size != p:
+        raise ValueError("shape mismatch")
+    if Y.size and (Y.min() < 0 or Y.max() > 1) or Z.size and (Z.min() < 0 or Z.max() > 1):
+        raise ValueError("Y and Z must hold 0 or 1")
+    W = np.empty((n, m), dtype=np.float64)
+    lib.oracle_bqq_dense_weight(_ptr(Y), _ptr(Z), _ptr(r), _ptr(s), _ptr(t), float(u), n, k, m, p, _ptr(W))
+    return W
+
+
+def bqq_forward(x, Y, Z, r, s, t, u) -> np.ndarray:
+    """y = x W^T for the BQQ weight W of bqq_dense_weight (x: batch x m)."""
+    return forward_dense(x, bqq_dense_weight(Y, Z, r, s, t, u))

@@ -35,8 +35,10 @@
  *
  * Parity status of each function (see the test-suite pins in
  * tests/test_oracle_pins.py):
- *   oracle_forward_staged, oracle_dense_weight, oracle_forward_dense,
- *   oracle_unpack_signs, oracle_pack_signs, oracle_bits_per_weight: pinned.
+ *   oracle_forward_staged, oracle_forward_transposed, oracle_dense_weight,
+ *   oracle_forward_dense, oracle_unpack_signs, oracle_pack_signs,
+ *   oracle_bits_per_weight, oracle_scale_bits_per_weight, oracle_bqq_dense_weight:
+ *   pinned.
  */
 #include <math.h>
 #include <stddef.h>
@@ -52,6 +54,15 @@ int oracle_num_threads(void) {
   return omp_get_max_threads();
 #else
   return 1;
+#endif
+}
+
+/* Threads for the parallel loops below (timing only; results do not depend on it). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
 #endif
 }
 
@@ -194,6 +205,43 @@ void oracle_dense_weight(const int8_t* A, const int8_t* B, const double* a, cons
       const double left = a[i] * (double)A[i * k + l] * mid[l];
       const int8_t* Bl = B + l * m_in;
       for (int64_t j = 0; j < m_in; ++j) Wi[j] += left * ((double)Bl[j] * b[j]);
+    }
+  }
+}
+
+/*
+ * Binary Quadratic Quantization (sciencestack.ai page of "Binary Quadratic
+ * Quantization: Beyond First-Order Quantization for Real-Valued Matrix
+ * Compression", TL;DR formula):
+ *     W = sum_{i<p} (r_i Y_i Z_i + s_i Y_i 1_Z + t_i 1_Y Z_i) + u 1,
+ * with binary Y_i (n x k) and Z_i (k x m), real scalars r_i, s_i, t_i, u, and
+ * 1_Z, 1_Y, 1 all-ones matrices of the shapes of Z_i, Y_i and W.  The binary
+ * alphabet is read as {0, 1} (the page builds on polynomial unconstrained
+ * binary optimisation).  Y holds the p matrices Y_i one after the other
+ * (p x n x k, row-major), Z likewise (p x k x m); entries 0 or 1.
+ *     (Y_i 1_Z)[a][c] = sum_l Y_i[a][l]       (1_Z is k x m)
+ *     (1_Y Z_i)[a][c] = sum_l Z_i[l][c]       (1_Y is n x k)
+ */
+void oracle_bqq_dense_weight(const int8_t* Y, const int8_t* Z, const double* r, const double* s, const double* t,
+                             double u, int64_t n, int64_t k, int64_t m, int64_t p, double* W) {
+#pragma omp parallel for schedule(static)
+  for (int64_t a = 0; a < n; ++a) {
+    for (int64_t c = 0; c < m; ++c) {
+      double w = u;
+      for (int64_t i = 0; i < p; ++i) {
+        const int8_t* Yi = Y + i * n * k;
+        const int8_t* Zi = Z + i * k * m;
+        double yz = 0.0, y_row = 0.0, z_col = 0.0;
+        for (int64_t l = 0; l < k; ++l) {
+          yz += (double)Yi[a * k + l] * (double)Zi[l * m + c];
+          y_row += (double)Yi[a * k + l];
+          z_col += (double)Zi[l * m + c];
+        }
+        w += r[i] * yz;
+        w += s[i] * y_row;
+        w += t[i] * z_col;
+      }
+      W[a * m + c] = w;
     }
   }
 }

@@ -2,7 +2,7 @@
 
 Each mutant is the oracle's C source with one edit (a dropped scale, a wrong
 sign, a transposed or reversed operand, a dropped term, a wrong bit layout,
-in the forward and in the transpose product),
+in the forward, the transpose product and the BQQ weight),
 compiled into a temporary library on the CPU.  The pins of
 test_oracle_pins.py are then run against the mutant; at least one must fail.
 This shows the pins are strong enough to trust the unmutated oracle.
@@ -14,6 +14,7 @@ import tempfile
 import pytest
 
 import oracle
+import test_oracle_bqq as bqq
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "dbf_oracle.c")
@@ -42,6 +43,15 @@ MUTANTS = {
                                      "acc += (double)A[l * n + i] * gbuf[i];"),
     "transposed_B_not_transposed": ("acc += (double)B[l * m_in + j] * vbuf[l];",
                                     "acc += (double)B[(j % k) * m_in + (l % m_in)] * vbuf[l];"),
+    "scale_bits_drop_mid": ("return 16.0 * (double)(n + k + m_in) / ((double)n * (double)m_in);",
+                            "return 16.0 * (double)(n + m_in) / ((double)n * (double)m_in);"),
+    "bqq_drops_s_term": ("        w += s[i] * y_row;\n", "        w += 0.0 * y_row;\n"),
+    "bqq_t_on_rows_of_Y": ("        w += t[i] * z_col;\n", "        w += t[i] * y_row;\n"),
+    "bqq_Z_transposed": ("          yz += (double)Yi[a * k + l] * (double)Zi[l * m + c];",
+                         "          yz += (double)Yi[a * k + l] * (double)Zi[(c % k) * m + (l % m)];"),
+    "bqq_u_dropped": ("      double w = u;", "      double w = 0.0;"),
+    "bqq_last_term_dropped": ("      for (int64_t i = 0; i < p; ++i) {\n        const int8_t* Yi",
+                              "      for (int64_t i = 0; i + 1 < p; ++i) {\n        const int8_t* Yi"),
     "bpw_off": ("return (double)k * (double)(n + m_in) / ((double)n * (double)m_in);",
                 "return (double)k * (double)(n + m_in) / ((double)n * (double)(m_in + 1));"),
 }
@@ -56,6 +66,7 @@ PIN_CHECKS = [
     lambda o: pins.test_k1_outer_product(o),
     lambda o: pins.test_orientation_is_not_transposed(o),
     lambda o: pins.test_bits_per_weight_closed_form(o, 4096, 2048, 4096, 1.0),
+    lambda o: pins.test_scale_bits_per_weight_counts_stored_vectors(o, 1024, 832, 4096),
     lambda o: pins.test_layout_table(o),
     lambda o: pins.test_layout_round_trip_and_padding(o, 3, 128),
     lambda o: pins.test_layout_hand_words(o),
@@ -64,6 +75,11 @@ PIN_CHECKS = [
     lambda o: pins.test_transposed_hadamard_closed_form(o, 3),
     lambda o: pins.test_transposed_integer_exact(o),
     lambda o: pins.test_transposed_uses_each_scale_once(o),
+    lambda o: bqq.test_bqq_hand_worked_example(o),
+    lambda o: bqq.test_bqq_product_term_is_integer_matmul(o, 16, 8, 33),
+    lambda o: bqq.test_bqq_all_ones_closed_form(o),
+    lambda o: bqq.test_bqq_reduces_to_dbf_weight(o, 3, 33, 24, 17),
+    lambda o: bqq.test_bqq_without_product_terms_has_rank_two(o),
 ]
 
 

@@ -242,7 +242,19 @@ def test_bits_per_weight_closed_form(oracle_mod, n, k, m_in, expect):
     if k % 256 == 0 and m_in % 256 == 0:
         words = n * oracle_mod.words_per_row(k) + k * oracle_mod.words_per_row(m_in)
         assert words * 32 / (n * m_in) == pytest.approx(expect, rel=1e-15)
-    assert oracle_mod.scale_bits_per_weight(n, k, m_in) == pytest.approx(16 * (n + k + m_in) / (n * m_in))
+
+
+@pytest.mark.parametrize("n,k,m_in", [(4096, 2048, 4096), (4096, 4096, 4096), (14336, 4736, 4096), (1024, 832, 4096),
+                                      (4096, 3200, 14336), (256, 128, 256), (3, 64, 5)])
+def test_scale_bits_per_weight_counts_stored_vectors(oracle_mod, n, k, m_in):
+    """The three scale vectors are stored as fp16 (sciencestack.ai Figure 1; gist.science section 2.1 names
+    a, m, b as FP16 vectors): their storage, counted from real fp16 arrays of lengths n, k and m_in,
+    spread over the n * m_in weights of the dense layer."""
+    rng = np.random.default_rng(n + k + m_in)
+    vecs = [gen.lognormal_scales(rng, n), gen.lognormal_scales(rng, k), gen.lognormal_scales(rng, m_in)]
+    assert all(v.dtype == np.float16 for v in vecs)
+    stored_bits = 8 * sum(v.nbytes for v in vecs)
+    assert oracle_mod.scale_bits_per_weight(n, k, m_in) == pytest.approx(stored_bits / (n * m_in), rel=1e-15)
 
 
 def test_bits_per_weight_rounding_rule():
