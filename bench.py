@@ -219,6 +219,21 @@ def oracle_rate(shape, batch, seconds, rotation=0):
     return batch * calls / el, calls, el, oracle.num_threads()
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+REFERENCE_MIN_SECONDS = 8.0
+
+
 def run_reference(args, shape, batch):
     world, rank, _ = dist_setup(args)
     if rank != 0:
@@ -229,15 +244,21 @@ def run_reference(args, shape, batch):
     oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])  # warm
     for _ in range(args.warmup):
         oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
+    # K steps of one layer forward each, continued until at least a few seconds
+    # are timed, so that the rate is stable whatever K the caller asks for
+    calls, t0 = 0, time.perf_counter()
+    while True:
         oracle.forward_staged(L["x"], L["A"], L["B"], L["a"], L["mid"], L["b"])
-    el = time.perf_counter() - t0
-    value = batch * args.steps / el
-    sample = f"one layer forward ({shape.name}, batch {batch}) per step out of the R-layer step of the GPU arm"
+        calls += 1
+        el = time.perf_counter() - t0
+        if calls >= args.steps and el >= REFERENCE_MIN_SECONDS:
+            break
+    value = batch * calls / el
+    sample = (f"{calls} fp64 oracle forwards of one {shape.name} layer at batch {batch} ({el:.1f} s; each the unit "
+              f"of the GPU arm's R-layer step); CPU: {cpu_model()}")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / calls,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(shape, batch), "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
@@ -278,8 +299,9 @@ class Workload:
         self.flags = dbf.DBF_FWD_WEIGHTS_STATIC if flags is None else flags
         self.weight_bytes_total = self.copies * weight_bytes
         decode = batch <= 16 and not (self.flags & dbf.DBF_FWD_FORCE_PREFILL)
-        self.launches_per_forward = 2 * (math.ceil(batch / 16) if decode else 1)
-        self.path = "decode (mma.sync sign-GEMV, 2 PDL-chained stages)" if decode else "prefill (tcgen05, 2 GEMMs)"
+        two_stage = self.flags & (dbf.DBF_FWD_DECODE_TWO_STAGE | dbf.DBF_FWD_DECODE_SHIFT_EXPAND)
+        self.launches_per_forward = ((1 if not two_stage else 2) * math.ceil(batch / 16)) if decode else 2
+        self.path = "decode" if decode else "prefill (tcgen05, 2 GEMMs)"
 
     def forward_all(self, x=None, y=None):
         x = self.x if x is None else x
@@ -364,6 +386,119 @@ class GroupWorkload(Workload):
             self.dbf.dbf_forward_grouped(self.x, grp, self.m_in, ys=self.ys, workspace=self.ws, flags=self.flags)
 
 
+def time_replays(torch, graph, reps, rounds=1):
+    """Device time (ms) of `reps` replays of a captured graph, CUDA events on
+    the current stream; the median over `rounds` rounds."""
+    times = []
+    for _ in range(rounds):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def path_name(wl, launches_per_layer):
+    if wl.batch <= 16 and not (wl.flags & wl.dbf.DBF_FWD_FORCE_PREFILL):
+        if launches_per_layer is not None and launches_per_layer <= math.ceil(wl.batch / 16):
+            return "decode: one launch per layer (int8 mma.sync sign products, V handed over inside the cluster)"
+        return "decode: two PDL-chained launches per layer (fp16 mma.sync sign-GEMV)"
+    return "prefill: tcgen05 GEMMs (two or three launches per layer)"
+
+
+def roofline_for(wl, shape, batch, us, peaks, traffic, peak_kind="burst"):
+    """The roofline object of one layer forward timed at `us` per layer."""
+    if batch > 16:
+        fl = layer_flops(shape.n, shape.k, shape.m_in, batch)
+        tf = fl / (us * 1e-6) / 1e12
+        peak = peaks["bf16_tflops"] if peak_kind == "burst" else peaks["bf16_tflops_sustained"]
+        return {"bound": "tensor", "kernel": "dbf_forward prefill (GEMM1 + GEMM2, one layer)", "achieved": tf,
+                "peak": peak, "unit": "TFLOP/s", "frac": tf / peak, "traffic": traffic,
+                "peak_source": f"{peaks['source']} dense bf16 {peak_kind} of measured (fp16 runs at the bf16 rate)",
+                "algorithmic_flops_per_layer": fl}
+    gbs = wl.bytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "kernel": "dbf_forward decode (one layer)", "achieved": gbs, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": traffic,
+            "peak_source": f"{peaks['source']} STREAM-style copy of measured (MEASURED_PEAKS.json)",
+            "algorithmic_bytes_per_layer": wl.bytes}
+
+
+def measure_workload(dbf, torch, shape, batch, device, peaks, rounds=5):
+    """One more configuration of the metric in the same run: R rotated copies in
+    one CUDA graph, device-timed; its own roofline."""
+    wl = Workload(dbf, torch, shape, batch, device)
+    g = wl.capture()
+    launches = graph_kernel_launches(g)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(3, int(400 / wl.copies))
+    ms = time_replays(torch, g, reps, rounds)
+    us = 1e3 * ms / reps / wl.copies
+    ok = dbf.dbf_workspace_status(wl.ws) == 0
+    out = {"workload": workload_name(shape, batch), "path": path_name(wl, None if launches is None else
+                                                                         launches / wl.copies),
+           "us_per_layer": us, "tokens_per_s": batch / (us * 1e-6), "layers_per_replay": wl.copies,
+           "launches_per_layer": None if launches is None else launches / wl.copies,
+           "roofline": roofline_for(wl, shape, batch, us, peaks, traffic_for(f"{shape.name}_b{batch}")),
+           "status_ok": ok}
+    del g, wl
+    torch.cuda.empty_cache()
+    return out
+
+
+def e2e_per_call(dbf, torch, wl, steps, warmup):
+    """End to end through the public C ABI, one call per layer: every step copies
+    x from pinned host memory, calls dbf_forward for each of the R layers (no
+    graph: the host cost of every call is inside the timed region) and reads y
+    back into pinned host memory.  Returns (tokens/s, h2d bytes, d2h bytes)."""
+    import ctypes
+
+    lib = dbf.load_library()
+    s = wl.shape
+    x_host = torch.from_numpy(np.ascontiguousarray(wl.host["x"])).pin_memory()
+    y_host = torch.empty((wl.batch, s.n), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty_like(wl.x)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = ctypes.c_void_p
+    ws_bytes = wl.ws.numel()
+    calls = []
+    for i in range(wl.copies):
+        a, mid, b = wl.sc[i]
+        calls.append((vp(x_dev.data_ptr()), vp(wl.pA[i].data_ptr()), vp(wl.pB[i].data_ptr()), vp(a.data_ptr()),
+                      vp(mid.data_ptr()), vp(b.data_ptr()), s.n, s.k, s.m_in, wl.batch, vp(wl.y.data_ptr()), 1,
+                      vp(wl.ws.data_ptr()), ws_bytes, wl.flags, sp))
+    fwd = lib.dbf_forward
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        bad = 0
+        for c in calls:
+            bad |= fwd(*c)
+        y_host.copy_(wl.y, non_blocking=True)
+        return bad
+
+    for _ in range(max(3, warmup)):
+        if step() != 0:
+            raise RuntimeError("dbf_forward failed in the end-to-end loop")
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    bad = 0
+    for _ in range(steps):
+        bad |= step()
+    e1.record()
+    torch.cuda.synchronize()
+    if bad != 0:
+        raise RuntimeError("dbf_forward failed in the end-to-end loop")
+    ms = e0.elapsed_time(e1)
+    return ms, int(x_host.numel() * 2), int(y_host.numel() * 2)
+
+
 def run_ours(args, shape, batch):
     import torch
 
@@ -426,40 +561,35 @@ def run_ours(args, shape, batch):
     tokens_per_s = whole_job_rate(batch * wl.copies * args.steps, world, ms)
     hbm_gbs = wl.bytes / (us_per_layer * 1e-6) / 1e9
 
-    # ---------------------------------------------------------- end to end: host buffers, copies inside
-    x_host = torch.from_numpy(np.ascontiguousarray(wl.host["x"])).pin_memory()
-    y_host = torch.empty((batch, shape.n), dtype=torch.float16).pin_memory()
-    x_dev = torch.empty_like(wl.x)
-    g2 = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        wl.forward_all(x=x_dev)
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    with torch.cuda.graph(g2):
-        wl.forward_all(x=x_dev)
-    torch.cuda.synchronize()
-    e2e_steps = max(1, args.steps)
-    for _ in range(max(3, args.warmup)):
-        x_dev.copy_(x_host, non_blocking=True)
-        g2.replay()
-        y_host.copy_(wl.y, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        g2.replay()
-        y_host.copy_(wl.y, non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    e2e_value = whole_job_rate(batch * wl.copies * e2e_steps, world, e2e_ms)
+    # cold single launch: one layer forward after writing a buffer of 2 x L2
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=device)
+    cold = []
+    for _ in range(5):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dbf.dbf_forward(wl.x, wl.pA[0], wl.pB[0], *wl.sc[0], shape.n, shape.k, shape.m_in, y=wl.y, workspace=wl.ws,
+                        flags=wl.flags)
+        e1.record()
+        torch.cuda.synchronize()
+        cold.append(1e3 * e0.elapsed_time(e1))
+    del flush
 
-    # output check of the timed configuration (sampled, against the oracle)
+    # ---------------------------------------------------------- end to end: host buffers, one C-ABI call per layer
+    e2e_steps = max(3, min(args.steps, 200))
+    e2e_ms, h2d, d2h = e2e_per_call(dbf, torch, wl, e2e_steps, args.warmup)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    e2e_value = whole_job_rate(batch * wl.copies * e2e_steps, world, e2e_ms)
+    status_ok = dbf.dbf_workspace_status(wl.ws) == 0
+
+    # the metric's other regimes in the same run (rank 0 reports them)
+    extra = []
+    if args.extra:
+        for name, b in (("mlp_up", 2048), ("attn_2b", 16)):
+            extra.append(measure_workload(dbf, torch, gen.CONFIGS[name], b, device, peaks))
+
+    # output check of the timed configuration (every token, against the oracle)
     check = None
     if rank == 0 and args.check:
         import oracle
@@ -467,12 +597,12 @@ def run_ours(args, shape, batch):
         torch.cuda.synchronize()
         ref = oracle.forward_staged(wl.host["x"], wl.host["A"], wl.host["B"], wl.host["a"], wl.host["mid"],
                                     wl.host["b"])
-        y = y_host.float().numpy().astype(np.float64)
+        y = wl.y.float().cpu().numpy().astype(np.float64)
         check = float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
 
     if world > 1:
         torch.distributed.barrier()
-        del graph, g2
+        del graph
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
@@ -480,13 +610,22 @@ def run_ours(args, shape, batch):
     # ---------------------------------------------------------- CPU baseline (oracle), rank 0 at N = 1 only
     cpu = None
     if world == 1 and args.cpu_seconds > 0:
+        import oracle
+
         rate, calls, el, cores = oracle_rate(shape, batch, args.cpu_seconds)
+        oracle.set_num_threads(1)
+        rate1, calls1, el1, _ = oracle_rate(shape, batch, max(1.0, args.cpu_seconds / 4))
+        oracle.set_num_threads(cores)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{calls} fp64 oracle forwards of one {shape.name} layer at batch {batch} "
-                         f"({el:.1f} s on host cores)"}
+                         f"({el:.1f} s on {cores} host threads)",
+               "one_thread": {"value": rate1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{calls1} forwards in {el1:.1f} s on one thread"},
+               "cpu_model": cpu_model()}
 
     key = f"{shape.name}_b{batch}"
     traffic = traffic_for(key)
+    launches_per_layer = step_launches / wl.copies
     result = {
         "metric": METRIC,
         "value": tokens_per_s,
@@ -502,7 +641,7 @@ def run_ours(args, shape, batch):
         "data": "synthetic",
         "config": {
             "workload": workload_name(shape, batch),
-            "path": wl.path,
+            "path": path_name(wl, launches_per_layer),
             "layers_per_step": wl.copies,
             "l2": f"inputs larger than L2: {wl.copies} distinct weight copies, "
                   f"{wl.weight_bytes_total / 1e6:.0f} MB >= 4 x L2",
@@ -510,34 +649,20 @@ def run_ours(args, shape, batch):
             "graph": "one CUDA graph of the step's dbf_forward calls, replayed once per step",
         },
         "us_per_layer": us_per_layer,
+        "us_cold_single_launch": statistics.median(cold),
         "hbm_gbs": hbm_gbs,
         "hbm_frac": hbm_gbs / peaks["hbm_gbs"],
-        "roofline": {
-            "bound": "hbm",
-            "kernel": "dbf_forward decode pair (stage B + stage A, PDL-overlapped, one layer)",
-            "achieved": hbm_gbs,
-            "peak": peaks["hbm_gbs"],
-            "unit": "GB/s",
-            "frac": hbm_gbs / peaks["hbm_gbs"],
-            "traffic": traffic,
-            "peak_source": f"{peaks['source']} (STREAM-style copy, MEASURED_PEAKS.json)",
-            "algorithmic_bytes_per_layer": wl.bytes,
-        },
+        "roofline": roofline_for(wl, shape, batch, us_per_layer, peaks, traffic),
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
-                "d2h_bytes_per_step": int(y_host.numel() * 2)},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": f"{e2e_steps} steps; per step: x from pinned host memory, {wl.copies} dbf_forward calls "
+                       "through the C ABI (ctypes, no graph), y back to pinned host memory; CUDA events"},
         "gpu_launches": args.steps * step_launches,
         "gpu_launches_source": launches_source,
         "clocks": clocks,
+        "workspace_status_ok": status_ok,
+        "also": extra,
     }
-    if batch > 16:
-        fl = layer_flops(shape.n, shape.k, shape.m_in, batch)
-        tf = fl / (us_per_layer * 1e-6) / 1e12
-        result["roofline"] = {
-            "bound": "tensor", "kernel": "dbf_forward prefill pair (GEMM1 + GEMM2, one layer)", "achieved": tf,
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "traffic": traffic,
-            "peak_source": f"{peaks['source']} dense bf16 burst (fp16 runs at the bf16 rate)",
-            "algorithmic_flops_per_layer": fl}
     if check is not None:
         result["output_check_rel_fro"] = check
     print(json.dumps(result))
@@ -698,6 +823,8 @@ def main():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-check", dest="check", action="store_false")
+    ap.add_argument("--no-extra", dest="extra", action="store_false",
+                    help="skip the batch-2048 and batch-16 configurations timed beside the main one")
     ap.add_argument("--sweep", default=None, help="run every config and write a JSON table here")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -25,13 +25,16 @@ __all__ = [
     "DBFError",
     "DBF_I8", "DBF_F16", "DBF_F32",
     "DBF_FWD_WEIGHTS_STATIC", "DBF_FWD_FORCE_DECODE", "DBF_FWD_FORCE_PREFILL", "DBF_FWD_DECODE_SHIFT_EXPAND",
+    "DBF_FWD_DECODE_TWO_STAGE", "DBF_FWD_DECODE_SINGLE", "DBF_FWD_TEST_LOSE_ARRIVAL",
     "EXPORTED_SYMBOLS",
     "library_path", "load_library",
     "dbf_packed_words_per_row", "dbf_packed_words", "dbf_pack_signs",
     "dbf_forward_workspace_bytes", "dbf_new_workspace", "dbf_forward",
     "dbf_reconstruct_dense", "dbf_workspace_status", "dbf_status_string", "dbf_forward_noalloc",
+    "dbf_noalloc_status",
     "DBF_MAX_GROUP", "dbf_forward_grouped_workspace_bytes", "dbf_new_grouped_workspace", "dbf_forward_grouped",
     "dbf_transpose_signs", "dbf_forward_transposed",
+    "dbf_bqq_prepared_bytes", "dbf_bqq_prepare", "dbf_bqq_workspace_bytes", "dbf_bqq_forward",
 ]
 
 DBF_I8, DBF_F16, DBF_F32 = 0, 1, 2
@@ -39,6 +42,9 @@ DBF_FWD_WEIGHTS_STATIC = 1 << 0
 DBF_FWD_FORCE_DECODE = 1 << 1
 DBF_FWD_FORCE_PREFILL = 1 << 2
 DBF_FWD_DECODE_SHIFT_EXPAND = 1 << 3
+DBF_FWD_DECODE_TWO_STAGE = 1 << 4
+DBF_FWD_DECODE_SINGLE = 1 << 5
+DBF_FWD_TEST_LOSE_ARRIVAL = 1 << 30  # test only: makes a bounded device wait run out
 
 STATUS_NAMES = {
     0: "DBF_OK", 1: "DBF_ERR_INVALID_ARG", 2: "DBF_ERR_UNSUPPORTED_SHAPE", 3: "DBF_ERR_MISALIGNED",
@@ -54,10 +60,15 @@ EXPORTED_SYMBOLS = (
     "dbf_reconstruct_dense",
     "dbf_workspace_status",
     "dbf_forward_noalloc",
+    "dbf_noalloc_status",
     "dbf_forward_grouped_workspace_bytes",
     "dbf_forward_grouped",
     "dbf_transpose_signs",
     "dbf_forward_transposed",
+    "dbf_bqq_prepared_bytes",
+    "dbf_bqq_prepare",
+    "dbf_bqq_workspace_bytes",
+    "dbf_bqq_forward",
     "dbf_status_string",
 )
 
@@ -112,6 +123,8 @@ def load_library():
     lib.dbf_workspace_status.restype = i32
     lib.dbf_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, u32, vp]
     lib.dbf_forward_noalloc.restype = i32
+    lib.dbf_noalloc_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.dbf_noalloc_status.restype = i32
     lib.dbf_forward_grouped_workspace_bytes.argtypes = [ctypes.POINTER(_LayerDesc), i32, i64, i64]
     lib.dbf_forward_grouped_workspace_bytes.restype = sz
     lib.dbf_forward_grouped.argtypes = [vp, i64, i64, ctypes.POINTER(_LayerDesc), i32, i32, vp, sz, u32, vp]
@@ -120,6 +133,14 @@ def load_library():
     lib.dbf_transpose_signs.restype = i32
     lib.dbf_forward_transposed.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, i32, vp, sz, u32, vp]
     lib.dbf_forward_transposed.restype = i32
+    lib.dbf_bqq_prepared_bytes.argtypes = [i64, i64, i64, i64]
+    lib.dbf_bqq_prepared_bytes.restype = sz
+    lib.dbf_bqq_prepare.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp, sz, vp]
+    lib.dbf_bqq_prepare.restype = i32
+    lib.dbf_bqq_workspace_bytes.argtypes = [i64, i64, i64, i64, i64]
+    lib.dbf_bqq_workspace_bytes.restype = sz
+    lib.dbf_bqq_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, i32, vp, sz, u32, vp]
+    lib.dbf_bqq_forward.restype = i32
     lib.dbf_status_string.argtypes = [i32]
     lib.dbf_status_string.restype = ctypes.c_char_p
     _LIB = lib
@@ -232,6 +253,13 @@ def dbf_forward_noalloc(x: torch.Tensor, packedA: torch.Tensor, packedB: torch.T
     return y
 
 
+def dbf_noalloc_status(stream=None) -> int:
+    """Status word of dbf_forward_noalloc's library buffer on the current device (synchronises the stream)."""
+    out = ctypes.c_int32(0)
+    _check("dbf_noalloc_status", load_library().dbf_noalloc_status(_stream(stream), ctypes.byref(out)))
+    return int(out.value)
+
+
 def dbf_reconstruct_dense(packedA: torch.Tensor, packedB: torch.Tensor, a: torch.Tensor, m: torch.Tensor,
                           b: torch.Tensor, n: int, k: int, m_in: int, W: Optional[torch.Tensor] = None,
                           W_dtype: torch.dtype = torch.float32, stream=None) -> torch.Tensor:
@@ -325,3 +353,35 @@ def dbf_forward_transposed(dy: torch.Tensor, packedAT: torch.Tensor, packedBT: t
         _ptr(dx), _dtype_code(dx.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(), int(flags),
         _stream(stream)))
     return dx
+
+
+def dbf_bqq_prepare(packedY: torch.Tensor, packedZ: torch.Tensor, r: torch.Tensor, s: torch.Tensor, t: torch.Tensor,
+                    u: torch.Tensor, n: int, k: int, p: int, m_in: int, stream=None) -> torch.Tensor:
+    """The weight-only part of the BQQ forward (mid, c, d); returns the prepared buffer (uint8 CUDA tensor)."""
+    nbytes = int(load_library().dbf_bqq_prepared_bytes(int(n), int(k), int(p), int(m_in)))
+    if nbytes == 0:
+        raise ValueError("shape outside the BQQ contract")
+    prep = torch.empty(nbytes, dtype=torch.uint8, device=packedY.device)
+    _check("dbf_bqq_prepare", load_library().dbf_bqq_prepare(
+        _ptr(packedY), _ptr(packedZ), _ptr(r), _ptr(s), _ptr(t), _ptr(u), int(n), int(k), int(p), int(m_in),
+        _ptr(prep), nbytes, _stream(stream)))
+    return prep
+
+
+def dbf_bqq_forward(x: torch.Tensor, packedY: torch.Tensor, packedZ: torch.Tensor, prepared: torch.Tensor, n: int,
+                    k: int, p: int, m_in: int, y: Optional[torch.Tensor] = None, y_dtype: torch.dtype = torch.float16,
+                    workspace: Optional[torch.Tensor] = None, flags: int = 0, stream=None) -> torch.Tensor:
+    """y = x W^T for the BQQ weight W = sum_i (r_i Y_i Z_i + s_i Y_i 1 + t_i 1 Z_i) + u 1; x fp16 batch x m_in."""
+    if x.dtype != torch.float16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp16 batch x m_in tensor")
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, n), dtype=y_dtype, device=x.device)
+    if workspace is None:
+        workspace = torch.zeros(int(load_library().dbf_bqq_workspace_bytes(int(n), int(k), int(p), int(m_in),
+                                                                           int(batch))),
+                                dtype=torch.uint8, device=x.device)
+    _check("dbf_bqq_forward", load_library().dbf_bqq_forward(
+        _ptr(x), _ptr(packedY), _ptr(packedZ), _ptr(prepared), int(n), int(k), int(p), int(m_in), int(batch),
+        _ptr(y), _dtype_code(y.dtype), _ptr(workspace), workspace.numel(), int(flags), _stream(stream)))
+    return y

@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdbf.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["dbf_api.cu", "decode.cu", "prefill.cu", "pack.cu", "transpose.cu", "reconstruct.cu", "noalloc.cu"]
+SOURCES = ["dbf_api.cu", "decode.cu", "fused.cu", "prefill.cu", "pack.cu", "transpose.cu", "reconstruct.cu", "bqq.cu", "noalloc.cu"]
 HEADERS = ["dbf_device.cuh", "dbf_internal.h"]
 
 NVCC_FLAGS = [

@@ -85,10 +85,26 @@ dbf_status dbf_pack_signs(const void* src, dbf_dtype src_t, int64_t rows, int64_
   return launch_pack(src, src_t, rows, cols, packed, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, int64_t batch) {
-  if (n < 1 || k < 1 || m_in < 1 || batch < 1) return 0;
+}  // extern "C"
+
+namespace {
+// Workspace layout: status block, V (batch x k fp16, the two-launch and
+// tensor-core paths), then the tagged partials of the single-launch decode
+// (batch x n x 8 64-bit words; only for batch <= 16).
+size_t v_area_end(int64_t k, int64_t batch) {
   const size_t v_bytes = static_cast<size_t>(batch) * static_cast<size_t>(k) * 2;
   return kStatusBytes + (v_bytes + 255) / 256 * 256;
+}
+size_t slot_bytes(int64_t n, int64_t tokens) {
+  return static_cast<size_t>(kFusedMaxSlices) * static_cast<size_t>(tokens) * static_cast<size_t>(n) * 8;
+}
+}  // namespace
+
+extern "C" {
+
+size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, int64_t batch) {
+  if (n < 1 || k < 1 || m_in < 1 || batch < 1) return 0;
+  return v_area_end(k, batch) + (batch <= 16 ? slot_bytes(n, batch) : 0);
 }
 
 static dbf_status validate_factors(const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
@@ -102,10 +118,12 @@ static dbf_status validate_factors(const uint32_t* packedA, const uint32_t* pack
   return DBF_OK;
 }
 
-dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
-                       const uint16_t* m, const uint16_t* b, int64_t n, int64_t k, int64_t m_in, int64_t batch,
-                       void* y, dbf_dtype y_t, void* workspace, size_t ws_bytes, uint32_t flags,
-                       struct CUstream_st* stream_handle) {
+}  // extern "C"
+
+namespace dbf {
+dbf_status validate_forward_args(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB,
+                                 const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n, int64_t k,
+                                 int64_t m_in, int64_t batch, const void* y, dbf_dtype y_t, uint32_t flags) {
   if (!x || !y) return DBF_ERR_INVALID_ARG;
   dbf_status st = validate_factors(packedA, packedB, a, m, b, n, k, m_in);
   if (st != DBF_OK) return st;
@@ -113,10 +131,25 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
   if (batch > kMaxRows) return DBF_ERR_UNSUPPORTED_SHAPE;
   if (y_t != DBF_F16 && y_t != DBF_F32) return DBF_ERR_INVALID_ARG;
   const uint32_t known = DBF_FWD_WEIGHTS_STATIC | DBF_FWD_FORCE_DECODE | DBF_FWD_FORCE_PREFILL |
-                         DBF_FWD_DECODE_SHIFT_EXPAND;
+                         DBF_FWD_DECODE_SHIFT_EXPAND | DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SINGLE |
+                         DBF_FWD_TEST_LOSE_ARRIVAL;
   if ((flags & ~known) != 0) return DBF_ERR_INVALID_ARG;
+  if ((flags & DBF_FWD_DECODE_SINGLE) && (flags & (DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SHIFT_EXPAND)))
+    return DBF_ERR_INVALID_ARG;
   if ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)) return DBF_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return DBF_ERR_MISALIGNED;
+  return DBF_OK;
+}
+}  // namespace dbf
+
+extern "C" {
+
+dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
+                       const uint16_t* m, const uint16_t* b, int64_t n, int64_t k, int64_t m_in, int64_t batch,
+                       void* y, dbf_dtype y_t, void* workspace, size_t ws_bytes, uint32_t flags,
+                       struct CUstream_st* stream_handle) {
+  dbf_status st = validate_forward_args(x, packedA, packedB, a, m, b, n, k, m_in, batch, y, y_t, flags);
+  if (st != DBF_OK) return st;
   if (!workspace || !aligned16(workspace) || ws_bytes < dbf_forward_workspace_bytes(n, k, m_in, batch))
     return DBF_ERR_WORKSPACE;
   DeviceInfo dev;
@@ -137,8 +170,36 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
   const bool decode = (flags & DBF_FWD_FORCE_DECODE) || (!(flags & DBF_FWD_FORCE_PREFILL) && batch <= 16);
   if (decode) {
     const bool class_expand = (flags & DBF_FWD_DECODE_SHIFT_EXPAND) == 0;
+    // the single-launch kernel when asked for (its measured per-layer time
+    // does not yet beat the two launches on any layer shape of the workloads)
+    const bool two_stage = (flags & DBF_FWD_DECODE_SINGLE) == 0;
     for (int64_t t0 = 0; t0 < batch; t0 += 16) {
       const int nb = static_cast<int>(batch - t0 < 16 ? batch - t0 : 16);
+      // one launch for the whole layer where the shape fits the kernel and the
+      // workspace has room for the cross-cluster partials
+      FusedArgs fa{};
+      size_t fsmem = 0;
+      if (!two_stage && plan_fused(n, k, m_in, nb, &fa, &fsmem) &&
+          ws_bytes >= v_area_end(k, batch) + slot_bytes(n, nb)) {
+        fa.x = xh + t0 * m_in;
+        fa.ld_x = m_in;
+        fa.packedB = packedB;
+        fa.wprB = words_per_row(m_in);
+        fa.packedA = packedA;
+        fa.wprA = words_per_row(k);
+        fa.a = ah;
+        fa.mid = mh;
+        fa.b = bh;
+        fa.y = static_cast<char*>(y) + static_cast<size_t>(t0) * static_cast<size_t>(n) * y_elt;
+        fa.ld_y = n;
+        fa.weights_early = early ? 1 : 0;
+        fa.test_lose_bytes = (flags & DBF_FWD_TEST_LOSE_ARRIVAL) ? 1 : 0;
+        fa.status = status;
+        fa.slots = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + v_area_end(k, batch));
+        st = launch_fused_decode(fa, fsmem, out_f32, stream);
+        if (st == DBF_OK) continue;
+        (void)cudaGetLastError();  // the launch was refused (e.g. no room for the cluster): two launches instead
+      }
       DecodeArgs sb{};
       sb.packed = packedB;
       sb.wpr = words_per_row(m_in);
@@ -235,8 +296,9 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
   if (batch < 1) return DBF_ERR_INVALID_ARG;
   if (batch > kMaxRows) return DBF_ERR_UNSUPPORTED_SHAPE;
   if (y_t != DBF_F16 && y_t != DBF_F32) return DBF_ERR_INVALID_ARG;
+  // (the grouped decode always runs the two-launch kernels: DBF_FWD_DECODE_TWO_STAGE changes nothing here)
   const uint32_t known = DBF_FWD_WEIGHTS_STATIC | DBF_FWD_FORCE_DECODE | DBF_FWD_FORCE_PREFILL |
-                         DBF_FWD_DECODE_SHIFT_EXPAND;
+                         DBF_FWD_DECODE_SHIFT_EXPAND | DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SINGLE;
   if ((flags & ~known) != 0) return DBF_ERR_INVALID_ARG;
   if ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)) return DBF_ERR_INVALID_ARG;
   if (!aligned16(x)) return DBF_ERR_MISALIGNED;

@@ -53,6 +53,12 @@ struct DeviceInfo {
 
 dbf_status current_device(DeviceInfo* info);
 
+// The synchronous argument checks of dbf_forward other than the workspace
+// (shared by every entry point that runs the layer forward).
+dbf_status validate_forward_args(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB,
+                                 const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n, int64_t k,
+                                 int64_t m_in, int64_t batch, const void* y, dbf_dtype y_t, uint32_t flags);
+
 dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
                                cudaStream_t stream);
 
@@ -72,6 +78,38 @@ struct DecodeGroup {
 // the forward's other stage (all layers).
 dbf_status launch_decode_group(DecodeGroup& group, int64_t peer_rows, bool class_expand, bool out_f32,
                                const DeviceInfo& dev, cudaStream_t stream);
+
+// The single-launch decode forward (fused.cu): grid (R, J), clusters of R
+// CTAs along x, one cluster per slice of kb middle rows.
+constexpr int kFusedMaxSlices = 8;
+struct FusedArgs {
+  const __half* x;
+  int64_t ld_x;
+  const uint32_t* packedB;  // k rows over m_in
+  int64_t wprB;
+  const uint32_t* packedA;  // n rows over k
+  int64_t wprA;
+  const __half* a;
+  const __half* mid;
+  const __half* b;
+  void* y;
+  int64_t ld_y;
+  int n, k, m_in, batch;     // batch 1..16
+  int MB;                    // 256-column blocks of m_in
+  int R;                     // CTAs per cluster (power of two <= 16)
+  int J;                     // clusters (slices of k)
+  int kb;                    // middle rows per slice (multiple of 256)
+  int nb;                    // output rows per rank (multiple of 16)
+  int weights_early;
+  int test_lose_bytes;       // test only: rank 0 waits for bytes that never come
+  int* status;
+  unsigned long long* slots; // batch x n x 8 tagged partials (word j - 1 from slice j)
+};
+
+// Fills the sizes of `args` for this shape; false if the shape does not fit
+// the single-launch kernel (then the two-launch path runs).
+bool plan_fused(int64_t n, int64_t k, int64_t m_in, int batch, FusedArgs* args, size_t* smem_bytes);
+dbf_status launch_fused_decode(const FusedArgs& args, size_t smem_bytes, bool out_f32, cudaStream_t stream);
 
 dbf_status launch_prefill_gemm(const PrefillArgs& args, const __half* act, int64_t act_rows, bool out_f32,
                                const DeviceInfo& dev, cudaStream_t stream);

@@ -41,6 +41,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "dbf_device.cuh"
 #include "dbf_internal.h"
@@ -57,6 +58,7 @@ constexpr int kDecThreads = 128;
 // while the previous group is multiplied)
 constexpr int kMaxClusterK = 8;
 constexpr int kSmemBudget = 100 * 1024;
+constexpr int kMaxDynSmem = 227 * 1024;  // opt-in limit of one CTA on sm_100
 constexpr int kHeadBytes = 512;  // mbarriers, abort flag, class sums and their per-warp parts
 
 // 1 / c_s for the class form: c_s is the fp16 value with only bit s set.
@@ -419,6 +421,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     pk = pe;
     if (pk >= k_hi) break;
     pe = min(k_hi, pk + piece);
+    // The next piece's bulk copies (async proxy) overwrite shared memory this
+    // piece wrote (the b-scaled activations) and read with ordinary accesses:
+    // order those accesses before the copies.
+    fence_proxy_async_smem();
     __syncthreads();  // everyone is done with this piece's activations and b
     slice(pk, pe, sb0, sb1);
     load_group(wa, sb0, sb1);
@@ -485,8 +491,14 @@ dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cu
   auto kernel = dbf_decode_stage_kernel<NT, RT, D, TOKPAR, CLASS, KSCALE, OUT_F32>;
   const DecSmem L = dec_smem_layout(piece, batch < NT * 8 ? batch : NT * 8, NT * 8, ks, RT);
   const size_t smem = static_cast<size_t>(L.total);
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (err != cudaSuccess) return DBF_ERR_CUDA;
+  // the shared-memory limit once per instantiation (the largest a CTA may ask for)
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  });
+  if (attr_err != cudaSuccess || smem > static_cast<size_t>(kMaxDynSmem)) return DBF_ERR_CUDA;
+  cudaError_t err;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grp.tile_start[grp.n]), static_cast<unsigned>(ks), 1);

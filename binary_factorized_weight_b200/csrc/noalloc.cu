@@ -12,11 +12,13 @@
 // Host code cannot use the array's name as a device address (on the host it
 // only names a shadow symbol), so the first call on each device, with that
 // device current, looks the address up with cudaGetSymbolAddress and caches
-// it; that first call should therefore come before any stream capture.  The
-// call itself allocates nothing: it clears the status word with
-// cudaMemsetAsync and hands the buffer to dbf_forward as its workspace.
-// Every call shares the one buffer, so calls whose work overlaps on the GPU
-// (different streams, or different host threads) race on it.
+// it; that first call should therefore come before any stream capture.  A
+// lookup that fails is not cached: the error it left is cleared and the next
+// call tries again.  The call itself allocates nothing: it clears the status
+// word with cudaMemsetAsync and hands the buffer to the forward as its
+// workspace.  dbf_noalloc_status reads that status word back.  Every call
+// shares the one buffer, so calls whose work overlaps on the GPU (different
+// streams, or different host threads) race on it.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -30,44 +32,23 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// Device address of the buffer on the current device `device` (cached after
+// the first successful lookup).
 void* scratch_address(int device, dbf_status* st) {
   static void* addr[kMaxDevices] = {};
-  static std::once_flag once[kMaxDevices];
-  static cudaError_t err[kMaxDevices] = {};
-  std::call_once(once[device], [device] {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[device] == nullptr) {
     void* p = nullptr;
-    err[device] = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // device `device` is current here
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();  // leave no sticky error for a later launch check
+      *st = DBF_ERR_CUDA;
+      return nullptr;
+    }
     addr[device] = p;
-  });
-  if (err[device] != cudaSuccess || addr[device] == nullptr) {
-    *st = DBF_ERR_CUDA;
-    return nullptr;
   }
   *st = DBF_OK;
   return addr[device];
-}
-
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// The synchronous argument checks dbf_forward makes, run before this entry
-// point enqueues its status-word clear, so that a rejected call enqueues nothing.
-dbf_status precheck(const uint16_t* x, const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
-                    const uint16_t* m, const uint16_t* b, int64_t n, int64_t k, int64_t m_in, int64_t batch,
-                    const void* y, dbf_dtype y_t, uint32_t flags) {
-  if (!x || !packedA || !packedB || !a || !m || !b || !y) return DBF_ERR_INVALID_ARG;
-  if (n < 1 || k < 1 || m_in < 1 || batch < 1) return DBF_ERR_INVALID_ARG;
-  if (k % 64 != 0 || m_in % 64 != 0 || k > (int64_t{1} << 20) || m_in > (int64_t{1} << 20) ||
-      n > (int64_t{1} << 24) || batch > (int64_t{1} << 24))
-    return DBF_ERR_UNSUPPORTED_SHAPE;
-  if (y_t != DBF_F16 && y_t != DBF_F32) return DBF_ERR_INVALID_ARG;
-  const uint32_t known = DBF_FWD_WEIGHTS_STATIC | DBF_FWD_FORCE_DECODE | DBF_FWD_FORCE_PREFILL |
-                         DBF_FWD_DECODE_SHIFT_EXPAND;
-  if ((flags & ~known) != 0 || ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)))
-    return DBF_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(packedA) || !aligned16(packedB) || !aligned16(a) || !aligned16(m) ||
-      !aligned16(b) || !aligned16(y))
-    return DBF_ERR_MISALIGNED;
-  return DBF_OK;
 }
 
 }  // namespace
@@ -78,7 +59,7 @@ dbf_status dbf_forward_noalloc(const uint16_t* x, const uint32_t* packedA, const
                                const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n, int64_t k,
                                int64_t m_in, int64_t batch, void* y, dbf_dtype y_t, uint32_t flags,
                                struct CUstream_st* stream) {
-  dbf_status st = precheck(x, packedA, packedB, a, m, b, n, k, m_in, batch, y, y_t, flags);
+  dbf_status st = dbf::validate_forward_args(x, packedA, packedB, a, m, b, n, k, m_in, batch, y, y_t, flags);
   if (st != DBF_OK) return st;
   if (dbf_forward_workspace_bytes(n, k, m_in, batch) > kNoAllocScratchBytes) return DBF_ERR_WORKSPACE;
   dbf::DeviceInfo dev;
@@ -92,6 +73,17 @@ dbf_status dbf_forward_noalloc(const uint16_t* x, const uint32_t* packedA, const
     return DBF_ERR_CUDA;
   return dbf_forward(x, packedA, packedB, a, m, b, n, k, m_in, batch, y, y_t, ws, kNoAllocScratchBytes, flags,
                      stream);
+}
+
+dbf_status dbf_noalloc_status(struct CUstream_st* stream, int32_t* device_status) {
+  if (!device_status) return DBF_ERR_INVALID_ARG;
+  dbf::DeviceInfo dev;
+  dbf_status st = dbf::current_device(&dev);
+  if (st != DBF_OK) return st;
+  if (dev.device >= kMaxDevices) return DBF_ERR_DEVICE;
+  void* ws = scratch_address(dev.device, &st);
+  if (st != DBF_OK) return st;
+  return dbf_workspace_status(ws, stream, device_status);
 }
 
 }  // extern "C"

@@ -562,8 +562,10 @@ dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, co
                         cudaStream_t stream) {
   auto kernel = dbf_prefill_gemm_kernel<NTILE, SPLIT, KSCALE, OUT_F32>;
   constexpr int smem = Cfg<NTILE, SPLIT>::kSmemBytes;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return DBF_ERR_CUDA;
+  static std::once_flag once;  // the attribute once per instantiation
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] { attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
+  if (attr_err != cudaSuccess) return DBF_ERR_CUDA;
   const int64_t m_tiles = (a.M + kBM - 1) / kBM;
   const int64_t n_tiles = (a.batch + NTILE - 1) / NTILE;
   // split K: one (tile, K slice) item per CTA, the ks slices of a tile in one cluster
@@ -596,6 +598,48 @@ dbf_status launch_split(const PrefillArgs& a, const CUtensorMap& map, int ks, bo
 }
 
 }  // namespace
+
+// The activation tensor map of one (pointer, K, rows, tile) on the current
+// device: encoded once and kept in a small table (a forward reuses the same
+// activation buffers call after call; encoding costs about a microsecond).
+static bool activation_map(const __half* act, int64_t K, int64_t rows, int ntile,
+                           PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* out) {
+  struct Entry {
+    const void* ptr;
+    int64_t K, rows;
+    int ntile, device;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 64;
+  static Entry table[kEntries];
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i) {
+    const Entry& e = table[i];
+    if (e.ptr == act && e.K == K && e.rows == rows && e.ntile == ntile && e.device == device) {
+      *out = e.map;
+      return true;
+    }
+  }
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(ntile)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(act), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return false;
+  Entry& e = table[next];
+  e = Entry{act, K, rows, ntile, device, map};
+  next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
+  *out = map;
+  return true;
+}
 
 // Tile shape and K split.  128 x 128 tiles with no split when there are enough
 // of them to occupy half the SMs (128 x 256 past 128 tokens); otherwise the K
@@ -689,14 +733,7 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
   }
 
   CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(act_rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(ntile)};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(act), dims, strides, box, estr,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return DBF_ERR_CUDA;
+  if (!activation_map(act, a.K, act_rows, ntile, encode, &map)) return DBF_ERR_CUDA;
 
   if (ks > 1) return launch_split<128, true>(a, map, ks, out_f32, dev, stream);
   if (ntile == 256) return launch_split<256, false>(a, map, 1, out_f32, dev, stream);

@@ -92,9 +92,25 @@ enum {
   DBF_FWD_FORCE_DECODE = 1u << 1,
   /* Force the tensor-core (tcgen05) path at any batch size. */
   DBF_FWD_FORCE_PREFILL = 1u << 2,
-  /* Decode path: form the fp16 sign operands by shift+mask with one
-   * accumulator set instead of the default bit-position classes. */
-  DBF_FWD_DECODE_SHIFT_EXPAND = 1u << 3
+  /* Two-launch decode path: form the fp16 sign operands by shift+mask with
+   * one accumulator set instead of the default bit-position classes (implies
+   * DBF_FWD_DECODE_TWO_STAGE). */
+  DBF_FWD_DECODE_SHIFT_EXPAND = 1u << 3,
+  /* Decode path: run the two products as two PDL-chained launches (fp16
+   * tensor-core sign-GEMV) instead of the single-launch kernel. */
+  DBF_FWD_DECODE_TWO_STAGE = 1u << 4,
+  /* Decode path: run the whole layer as one launch (int8 tensor-core sign
+   * products in block fixed point, the middle vector exchanged inside
+   * thread-block clusters) wherever the shape fits it, instead of the
+   * library's choice between the two decode kernels. */
+  DBF_FWD_DECODE_SINGLE = 1u << 5,
+  /* TEST ONLY.  Makes one bounded wait of the single-launch decode kernel run
+   * out (rank 0 of each cluster waits for 16 bytes that are never sent), so
+   * that failure reporting can be tested without a fault: the call still
+   * returns DBF_OK, the kernel ends after the wait budget (about 0.2-0.4 s)
+   * with y unwritten, and the workspace status word reads DBF_ERR_TIMEOUT.
+   * The workspace must then be zero-filled again before its next use. */
+  DBF_FWD_TEST_LOSE_ARRIVAL = 1u << 30
 };
 
 /* Words (uint32) in one packed row of `cols` signs: ceil(cols/256)*8.
@@ -192,10 +208,14 @@ DBF_API dbf_status dbf_workspace_status(const void* workspace, struct CUstream_s
  * in the library (a static __device__ array, held by every GPU that loads the
  * library until the process exits).  It allocates and frees nothing.
  *   Limit: dbf_forward_workspace_bytes(n, k, m_in, batch) <= 2 MiB, i.e.
- *   256 + batch*k*2 bytes (e.g. batch 16 with k up to 65528, or batch 256 with
- *   k up to 4095); larger sizes return DBF_ERR_WORKSPACE.
+ *   256 + batch*k*2 bytes (e.g. batch 16 with k up to 65472, or batch 256 with
+ *   k up to 4032, k being a multiple of 64); larger sizes return
+ *   DBF_ERR_WORKSPACE.
  *   The first call on each device looks up the buffer's device address with
- *   that device current; make that first call before any stream capture.
+ *   that device current; make that first call before any stream capture.  A
+ *   failed lookup (DBF_ERR_CUDA) is not remembered: the next call retries.
+ *   Device-side failures (a bounded wait that gave up) are read back with
+ *   dbf_noalloc_status.
  *   Each call clears the buffer's status word (cudaMemsetAsync on `stream`)
  *   before its kernels; the buffer keeps the last call's other contents.
  *   All calls share the one buffer: calls whose work overlaps on the GPU
@@ -206,6 +226,17 @@ DBF_API dbf_status dbf_forward_noalloc(const uint16_t* x, const uint32_t* packed
                                        const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n,
                                        int64_t k, int64_t m_in, int64_t batch, void* y, dbf_dtype y_t,
                                        uint32_t flags, struct CUstream_st* stream);
+
+/*
+ * The status word of dbf_forward_noalloc's library buffer on the current
+ * device, copied to *device_status (synchronises `stream`): 0 if the last
+ * dbf_forward_noalloc call's kernels (the word is cleared at each call) saw
+ * no device-side wait give up, else the dbf_status of the first failure
+ * (DBF_ERR_TIMEOUT).  Like dbf_forward_noalloc it allocates nothing; its first
+ * use on a device looks the buffer up as described there.  (No counterpart
+ * in the pages: it reports on the library's own buffer.)
+ */
+DBF_API dbf_status dbf_noalloc_status(struct CUstream_st* stream, int32_t* device_status);
 
 /*
  * Several layers that read the same input x: the same computation as one
@@ -280,6 +311,46 @@ DBF_API dbf_status dbf_forward_transposed(const uint16_t* dy, const uint32_t* pa
                                           int64_t k, int64_t m_in, int64_t batch, void* dx, dbf_dtype dx_t,
                                           void* workspace, size_t ws_bytes, uint32_t flags,
                                           struct CUstream_st* stream);
+
+/*
+ * Binary Quadratic Quantization (BQQ) forward, on the sign-product kernels.
+ * The sciencestack.ai page of "Binary Quadratic Quantization: Beyond
+ * First-Order Quantization for Real-Valued Matrix Compression" (TL;DR) writes
+ * a compressed n x m_in matrix as
+ *     W = sum_{i<p} (r_i Y_i Z_i + s_i Y_i 1_Z + t_i 1_Y Z_i) + u 1
+ * with binary Y_i (n x k) and Z_i (k x m_in) and all-ones matrices 1_Z, 1_Y, 1
+ * of the shapes of Z_i, Y_i and W.  The binary entries are read as {0, 1}.
+ * y = x W^T is evaluated as one DBF product plus a rank-two correction:
+ *     y = S_Y diag(r_i / 4 per term) S_Z x + c (1^T x) + 1 (d^T x),
+ * S_Y = 1 - 2 [Y_0 .. Y_p-1] and S_Z = 1 - 2 [Z_0; ..; Z_p-1] as sign matrices,
+ * c = sum_i (s_i + r_i/2) rowsum(Y_i), d = sum_i (t_i + r_i/2) colsum(Z_i)
+ * + u - k sum_i r_i / 4 (exact algebra; no approximation).
+ *
+ *   packedY    [Y_0 .. Y_{p-1}] side by side, n rows over p*k columns, in the
+ *              packed layout with a set bit for each 1 (dbf_pack_signs of
+ *              1 - 2Y, or of -Y).
+ *   packedZ    [Z_0; ..; Z_{p-1}] stacked, p*k rows over m_in columns, likewise.
+ *   r, s, t    p fp16 scalars each; u one fp16 scalar (device pointers).
+ *   prepared   dbf_bqq_prepared_bytes(...) bytes, written by dbf_bqq_prepare:
+ *              mid = r_i / 4 (p*k fp16), a vector of ones, c (n fp32) and
+ *              d (m_in fp32).  It depends on the weights only: prepare once.
+ * Shape contract: p*k and m_in multiples of 64 in [64, 1 << 20]; n and batch
+ * in [1, 1 << 24]; p <= 4096.  Pointers 16-byte aligned.
+ * dbf_bqq_forward: x batch x m_in fp16, y batch x n (y_t DBF_F16 or DBF_F32),
+ * workspace >= dbf_bqq_workspace_bytes(...) zero-filled before its first use;
+ * flags as dbf_forward.  Arithmetic: the product term as dbf_forward (fp32
+ * accumulation), the correction in fp32, one rounding to y_t.
+ */
+DBF_API size_t dbf_bqq_prepared_bytes(int64_t n, int64_t k, int64_t p, int64_t m_in);
+DBF_API dbf_status dbf_bqq_prepare(const uint32_t* packedY, const uint32_t* packedZ, const uint16_t* r,
+                                   const uint16_t* s, const uint16_t* t, const uint16_t* u, int64_t n, int64_t k,
+                                   int64_t p, int64_t m_in, void* prepared, size_t prepared_bytes,
+                                   struct CUstream_st* stream);
+DBF_API size_t dbf_bqq_workspace_bytes(int64_t n, int64_t k, int64_t p, int64_t m_in, int64_t batch);
+DBF_API dbf_status dbf_bqq_forward(const uint16_t* x, const uint32_t* packedY, const uint32_t* packedZ,
+                                   const void* prepared, int64_t n, int64_t k, int64_t p, int64_t m_in, int64_t batch,
+                                   void* y, dbf_dtype y_t, void* workspace, size_t ws_bytes, uint32_t flags,
+                                   struct CUstream_st* stream);
 
 /* Static, NUL-terminated description of a status code. */
 DBF_API const char* dbf_status_string(dbf_status status);

@@ -56,9 +56,12 @@ def test_packed_words(lib):
 
 
 def test_workspace_bytes(lib):
-    assert dbf.dbf_forward_workspace_bytes(4096, 2048, 4096, 1) == 256 + 4096
-    assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 4) == 256 + 1024
-    assert dbf.dbf_forward_workspace_bytes(256, 64, 256, 1) == 256 + 256  # V padded to 256 bytes
+    # status block + V (batch x k fp16, padded to 256 bytes) + for batch <= 16 the
+    # single-launch decode's tagged partials: batch x n x 8 words of 8 bytes
+    assert dbf.dbf_forward_workspace_bytes(4096, 2048, 4096, 1) == 256 + 4096 + 8 * 4096 * 8
+    assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 4) == 256 + 1024 + 8 * 4 * 256 * 8
+    assert dbf.dbf_forward_workspace_bytes(256, 64, 256, 1) == 256 + 256 + 8 * 256 * 8
+    assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 17) == 256 + 17 * 256  # no partials past 16 tokens
     assert dbf.dbf_forward_workspace_bytes(0, 128, 256, 4) == 0
 
 
@@ -87,7 +90,8 @@ def fwd(lib, x=P, A=P, B=P, a=P, m=P, b=P, n=256, k=128, m_in=256, batch=4, y=P,
         (dict(k=96), SHAPE), (dict(m_in=100), SHAPE), (dict(k=1 << 21), SHAPE), (dict(n=(1 << 24) + 1), SHAPE),
         (dict(batch=(1 << 24) + 1), SHAPE),
         (dict(y_t=0), INVALID), (dict(y_t=7), INVALID),
-        (dict(flags=1 << 9), INVALID), (dict(flags=2 | 4), INVALID),
+        (dict(flags=1 << 9), INVALID), (dict(flags=2 | 4), INVALID), (dict(flags=32 | 16), INVALID),
+        (dict(flags=32 | 8), INVALID),
         (dict(x=MIS), MISALIGNED), (dict(A=MIS), MISALIGNED), (dict(B=MIS), MISALIGNED),
         (dict(a=MIS), MISALIGNED), (dict(y=MIS), MISALIGNED),
         (dict(ws=None), WORKSPACE), (dict(ws=MIS), WORKSPACE), (dict(ws_bytes=256 + 1023), WORKSPACE),

@@ -26,11 +26,11 @@ def test_every_entry_names_its_sources():
         assert per_kernel == entry["dram_bytes_per_forward"], key
 
 
-def test_bench_workload_traffic_is_current():
-    # the default bench line (decode, attn_1b at batch 1) quotes the committed capture
-    entry = _entries()["attn_1b_b1"]
-    assert entry["source_hash"] == bench.kernel_source_hash(entry["source_files"])
-    assert bench.traffic_for("attn_1b_b1") == entry["dram_bytes_per_forward"]
+def test_bench_quotes_a_figure_only_for_current_sources():
+    # every committed figure is quoted while its sources are unchanged, and never after
+    for key, entry in _entries().items():
+        current = entry["source_hash"] == bench.kernel_source_hash(entry["source_files"])
+        assert bench.traffic_for(key) == (entry["dram_bytes_per_forward"] if current else None), key
 
 
 def test_changed_sources_void_the_figure(tmp_path, monkeypatch):

@@ -1,8 +1,7 @@
 """Parity of the configuration bench.py times: R rotated weight copies of a layer
 captured as one CUDA graph with DBF_FWD_WEIGHTS_STATIC (programmatic dependent
 launch chaining every forward), at the full sizes of the workloads.  The
-output after a replay is checked against the fp64 oracle on sampled tokens
-(every token for decode batches)."""
+output after a replay is checked against the fp64 oracle on every token."""
 import numpy as np
 import pytest
 import torch
@@ -33,10 +32,8 @@ def test_bench_launch_configuration(name, batch):
     torch.cuda.synchronize()
     assert dbf.dbf_workspace_status(wl.ws) == 0
     y = wl.y.float().cpu().numpy().astype(np.float64)
-    rows = np.arange(batch) if batch <= 16 else np.array([0, 1, 511, 1024, batch - 1])
-    ref = oracle.forward_staged(wl.host["x"][rows], wl.host["A"], wl.host["B"], wl.host["a"], wl.host["mid"],
-                                wl.host["b"])
-    got = y[rows]
+    ref = oracle.forward_staged(wl.host["x"], wl.host["A"], wl.host["B"], wl.host["a"], wl.host["mid"], wl.host["b"])
+    got = y  # every token
     assert np.all(np.isfinite(got))
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel <= 2e-3, rel

@@ -94,7 +94,9 @@ def test_grouped_single_layer_equals_forward(dbf):
     xd = dev(x)
     (yg,) = dbf.dbf_forward_grouped(xd, layers, 256)
     L = layers[0]
-    y1 = dbf.dbf_forward(xd, L["packedA"], L["packedB"], L["a"], L["m"], L["b"], L["n"], L["k"], 256)
+    # the grouped decode runs the two-launch kernels: the same arithmetic as dbf_forward's two-launch path
+    y1 = dbf.dbf_forward(xd, L["packedA"], L["packedB"], L["a"], L["m"], L["b"], L["n"], L["k"], 256,
+                         flags=dbf.DBF_FWD_DECODE_TWO_STAGE)
     torch.cuda.synchronize()
     assert torch.equal(yg, y1)
 

@@ -62,6 +62,9 @@ def test_noalloc_matches_workspace_forward_twice(lib, config, batch, y_dtype):
             assert np.array_equal(yn, rn)
         else:
             assert np.linalg.norm(yn - rn) / np.linalg.norm(rn) <= REL_FRO
+        status = ctypes.c_int32(-1)
+        assert c.dbf_noalloc_status(stream, ctypes.byref(status)) == 0
+        assert status.value == 0  # no device-side wait gave up
 
 
 def test_noalloc_rejects_sizes_beyond_its_buffer(lib):
