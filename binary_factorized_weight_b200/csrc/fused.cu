@@ -152,24 +152,26 @@ __device__ __forceinline__ float pow2f(int v) { return __int_as_float((v + 127) 
 
 // Block fixed point of the activations of one product, for this CTA's slice:
 // U[tok][0..cols) fp32 (zero past the valid columns) -> digit bytes in the MMA
-// order, per-token exponents exps[tok] and the digit sums of each token split
-// over the warps that built them: qpart[tok][part][d] (sum over part < wpt).
-// wpt = kFWarps / batch warps share a token (one warp per token past 8
-// tokens; warp w then also takes token w + 8), each taking every wpt-th run of
-// 32 columns.  One block barrier inside (the token maxima).
-__device__ __forceinline__ int warps_per_token(int batch) { return batch >= kFWarps ? 1 : kFWarps / batch; }
+// order, per-token exponents exps[tok] and the digit sums Q[3 tok + d].
+// 2^lg = kFWarps / batch warps share a token (one warp per token past 4
+// tokens; warp w then also takes token w + 8), each taking every 2^lg-th run
+// of 32 columns.  Two block barriers inside; Q is complete after the caller's
+// next barrier.
+__device__ __forceinline__ int warps_per_token_log2(int batch) { return batch == 1 ? 3 : batch == 2 ? 2 : batch <= 4 ? 1 : 0; }
 
 template <int NTILE>
-__device__ __noinline__ void build_digits(const float* U, int cols, int batch, uint8_t* dig, int* exps, int* qpart,
+__device__ __forceinline__ void build_digits(const float* U, int cols, int batch, uint8_t* dig, int* exps, int* Q,
                                           float* redmax) {
   constexpr int NCOL = 8 * NTILE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wpt = warps_per_token(batch);
-  const int part = warp % wpt;
-  const int tok0 = warp / wpt;
-  const int stride = 32 * wpt;
+  const int lg = warps_per_token_log2(batch);
+  const int part = warp & ((1 << lg) - 1);
+  const int tok0 = warp >> lg;
+  const int tstep = kFWarps >> lg;  // tokens handled by one pass of all warps
+  const int stride = 32 << lg;
+  if (threadIdx.x < 3 * kMaxTok) Q[threadIdx.x] = 0;
   // token maxima: each warp over its columns, then across the token's warps
-  for (int tok = tok0, slot = 0; tok < batch && tok0 < (kFWarps / wpt); tok += kFWarps / wpt, ++slot) {
+  for (int tok = tok0; tok < batch; tok += tstep) {
     const float* u = U + tok * cols;
     float mx = 0.f;
     for (int col = part * 32 + lane; col < cols; col += stride) mx = fmaxf(mx, fabsf(u[col]));
@@ -178,9 +180,13 @@ __device__ __noinline__ void build_digits(const float* U, int cols, int batch, u
     if (lane == 0) redmax[tok * kFWarps + part] = mx;
   }
   __syncthreads();
-  for (int tok = tok0; tok < batch && tok0 < (kFWarps / wpt); tok += kFWarps / wpt) {
+  for (int tok = tok0; tok < batch; tok += tstep) {
+    // the token's maximum from its warps' parts (all 8 slots read at once; unused ones are never 0-valued reads
+    // of other tokens because only 2^lg of them are combined)
     float mx = 0.f;
-    for (int q = 0; q < wpt; ++q) mx = fmaxf(mx, redmax[tok * kFWarps + q]);
+#pragma unroll
+    for (int q = 0; q < kFWarps; ++q)
+      if (q < (1 << lg)) mx = fmaxf(mx, redmax[tok * kFWarps + q]);
     // |q| < 2^22: e = 21 - floor(log2(max)), clamped so that 2^e stays a normal float
     int e = 0;
     if (mx > 0.f) {
@@ -216,20 +222,11 @@ __device__ __noinline__ void build_digits(const float* U, int cols, int batch, u
     }
     if (lane == 0) {
       if (part == 0) exps[tok] = e;
-      int* qp = qpart + (tok * kFWarps + part) * 3;
-      qp[0] = q0;
-      qp[1] = q1;
-      qp[2] = q2;
+      atomicAdd(&Q[3 * tok + 0], q0);  // integer sums: the order does not matter
+      atomicAdd(&Q[3 * tok + 1], q1);
+      atomicAdd(&Q[3 * tok + 2], q2);
     }
   }
-}
-
-// Digit sum of MMA column col (= 3 tok + d) from the per-warp parts.
-__device__ __forceinline__ int digit_sum(const int* qpart, int col, int wpt) {
-  const int tok = col / 3, d = col - 3 * tok;
-  int s = 0;
-  for (int q = 0; q < wpt; ++q) s += qpart[(tok * kFWarps + q) * 3 + d];
-  return s;
 }
 
 // One product over this CTA's tiles: out[tok][row] (fp32, rows of the tiles)
@@ -237,22 +234,18 @@ __device__ __forceinline__ int digit_sum(const int* qpart, int col, int wpt) {
 // int32 per digit, then 2^-e[tok] * (T2 * 65536 + T1 * 256 + T0).
 // w: weight items [tile][blk] of 16 rows x 32 bytes.  Warp w takes tiles w, w + 8, ...
 template <int NTILE, bool CLASS>
-__device__ __noinline__ void sign_product(const uint8_t* w, int tiles, int nblk, const uint8_t* dig, const int* exps,
-                                          const int* qpart, int batch, int* Tb, float* out, int ld_out) {
+__device__ __forceinline__ void sign_product(const uint8_t* w, int tiles, int nblk, const uint8_t* dig, const int* exps,
+                                          const int* Q, int batch, int* Tb, float* out, int ld_out) {
   constexpr int NCOL = 8 * NTILE;
   constexpr int NACC = CLASS ? 8 : 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   int* T = Tb + warp * 16 * NCOL;
-  const int wpt = warps_per_token(batch);
-  int qcol[NTILE][2];  // digit sums of this lane's columns
+  int qcol[NTILE][2];  // digit sums of this lane's columns (unused columns: anything)
 #pragma unroll
   for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int col = nt * 8 + 2 * c + h;
-      qcol[nt][h] = col < 3 * batch ? digit_sum(qpart, col, wpt) : 0;
-    }
+    for (int h = 0; h < 2; ++h) qcol[nt][h] = Q[nt * 8 + 2 * c + h];
   for (int t = warp; t < tiles; t += kFWarps) {
     int acc[NACC][NTILE][4];
 #pragma unroll
@@ -278,6 +271,38 @@ __device__ __noinline__ void sign_product(const uint8_t* w, int tiles, int nblk,
           mma_s8(acc[CLASS ? s : 0][nt], a0, a1, a2, a3, bf.x, bf.y);
         }
       }
+    }
+    if constexpr (NTILE == 1) {
+      // One N tile (batch <= 2): token t's digit columns 3t..3t+2 lie in lanes
+      // c = t and c + 1 of the quad, so the combination stays in registers.
+      int T[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int bits;
+        if constexpr (CLASS) {
+          bits = -(acc[7][0][e] >> 7);
+#pragma unroll
+          for (int s = 0; s < 7; ++s) bits += acc[s][0][e] >> s;
+        } else {
+          bits = acc[0][0][e];
+        }
+        T[e] = qcol[0][e & 1] - 2 * bits;
+      }
+      int Tn[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) Tn[e] = __shfl_down_sync(0xffffffffu, T[e], 1);
+      if (c < batch) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {  // rows g and g + 8
+          const int e0 = 2 * hr;
+          const int d0 = c == 0 ? T[e0] : T[e0 + 1];
+          const int d1 = c == 0 ? T[e0 + 1] : Tn[e0];
+          const int d2 = c == 0 ? Tn[e0] : Tn[e0 + 1];
+          const long long v = static_cast<long long>(d2) * 65536ll + static_cast<long long>(d1) * 256ll + d0;
+          out[c * ld_out + t * 16 + g + 8 * hr] = __ll2float_rn(v) * pow2f(-exps[c]);  // one rounding, exact scaling
+        }
+      }
+      continue;
     }
     // T = Q - 2 sum(bit * q) for rows g, g + 8 and columns 2c, 2c + 1 of each N tile
 #pragma unroll
@@ -318,7 +343,7 @@ __global__ void __launch_bounds__(kFThreads, 2) dbf_decode_fused_kernel(const __
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16);
   int* exps = reinterpret_cast<int*>(smem + 64);      // [16]
   float* redmax = reinterpret_cast<float*>(smem + 128);  // [16 tokens][8 warps]
-  int* qpart = reinterpret_cast<int*>(smem + 640);     // [16 tokens][8 warps][3 digits]
+  int* Q = reinterpret_cast<int*>(smem + 640);         // [48]: digit sums of the MMA columns
   uint8_t* wB = smem + L.wB;
   uint8_t* wA = smem + L.wA;
   uint8_t* dig = smem + L.dig;
@@ -426,12 +451,12 @@ __global__ void __launch_bounds__(kFThreads, 2) dbf_decode_fused_kernel(const __
     }
   }
   __syncthreads();
-  build_digits<NTILE>(U, colsB, batch, dig, exps, qpart, redmax);
+  build_digits<NTILE>(U, colsB, batch, dig, exps, Q, redmax);
   cp_async_wait_all();
   __syncthreads();
 
   // ---- first product: partial t of the slice's rows over this rank's columns
-  sign_product<NTILE, CLASS>(wB, tilesB, nblkB, dig, exps, qpart, batch, Tb, part, p.kb);
+  sign_product<NTILE, CLASS>(wB, tilesB, nblkB, dig, exps, Q, batch, Tb, part, p.kb);
   __syncthreads();
 
   // ---- V = mid (.) t for the slice, assembled in every rank of the cluster and
@@ -527,9 +552,9 @@ __global__ void __launch_bounds__(kFThreads, 2) dbf_decode_fused_kernel(const __
 
   // ---- second product: partial z of this rank's output rows over the slice
   if (tilesA > 0) {
-    build_digits<NTILE>(U, colsA, batch, dig, exps, qpart, redmax);
+    build_digits<NTILE>(U, colsA, batch, dig, exps, Q, redmax);
     __syncthreads();
-    sign_product<NTILE, CLASS>(wA, tilesA, nblkA, dig, exps, qpart, batch, Tb, zb, p.nb);
+    sign_product<NTILE, CLASS>(wA, tilesA, nblkA, dig, exps, Q, batch, Tb, zb, p.nb);
   }
   __syncthreads();
   if (rowsA == 0) return;
