@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload attn_1b] [--batch 1] [--sweep OUT.json]
+                    [--profile-calls N [--flags F]]   (plain calls for ncu captures)
 
 Workload (default): the Llama-8B-shaped attention projection n = m_in = 4096,
 k = 2048 (1.0 bit/weight), batch 1 (config attn_1b of dbf_inputs).  A step is
@@ -813,6 +814,33 @@ def run_sweep(args):
         json.dump({"peaks": peaks, "rows": rows}, f, indent=1)
 
 
+def run_profile_calls(args, shape, batch):
+    """For ncu captures: `--profile-calls N` plain dbf_forward calls of one layer
+    (no graph, no timing), with the given flags; exits non-zero on a wrong status."""
+    import torch
+
+    torch.cuda.set_device(0)
+    from binary_factorized_weight_b200 import build as lib_build
+
+    lib_build.build()
+    import binary_factorized_weight_b200 as dbf
+
+    dbf.load_library()
+    L = gen.make_layer(shape, batch)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    pA, pB = dbf.dbf_pack_signs(d(L["A"])), dbf.dbf_pack_signs(d(L["B"]))
+    a, mid, b, x = d(L["a"]), d(L["mid"]), d(L["b"]), d(L["x"])
+    ws = dbf.dbf_new_workspace(shape.n, shape.k, shape.m_in, batch)
+    y = None
+    for _ in range(args.profile_calls):
+        y = dbf.dbf_forward(x, pA, pB, a, mid, b, shape.n, shape.k, shape.m_in, workspace=ws, flags=args.flags)
+    torch.cuda.synchronize()
+    if dbf.dbf_workspace_status(ws) != 0:
+        raise SystemExit("device status word set")
+    print(json.dumps({"profile_calls": args.profile_calls, "workload": workload_name(shape, batch), "flags": args.flags,
+                      "mean_abs_y": float(y.float().abs().mean())}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -826,11 +854,16 @@ def main():
     ap.add_argument("--no-extra", dest="extra", action="store_false",
                     help="skip the batch-2048 and batch-16 configurations timed beside the main one")
     ap.add_argument("--sweep", default=None, help="run every config and write a JSON table here")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="only run this many dbf_forward calls of one layer (for ncu captures)")
+    ap.add_argument("--flags", type=int, default=1, help="dbf_forward flags for --profile-calls (default: weights static)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     shape = gen.CONFIGS[args.workload]
-    if args.sweep:
+    if args.profile_calls > 0:
+        run_profile_calls(args, shape, args.batch)
+    elif args.sweep:
         run_sweep(args)
     elif args.impl == "reference":
         run_reference(args, shape, args.batch)
