@@ -841,6 +841,55 @@ def run_profile_calls(args, shape, batch):
                       "mean_abs_y": float(y.float().abs().mean())}))
 
 
+def run_factorize(args):
+    """Offline factorisation timing: one 4096 x 4096 fp32 weight (Gaussian, column
+    scales falling from 2 to 0.2), k from --fact-k, the start and --fact-passes
+    alternating passes of 20 ADMM steps per factor, each pass timed with CUDA
+    events.  Dense products are cuBLAS SGEMM (fp32): the flops of one pass are
+    counted as its GEMMs' 2*M*N*K and reported against the fp32 rate."""
+    import torch
+
+    torch.cuda.set_device(0)
+    from binary_factorized_weight_b200 import build as lib_build
+
+    lib_build.build()
+    import binary_factorized_weight_b200 as dbf
+
+    dbf.load_library()
+    n = m = 4096
+    k = args.fact_k
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((n, m)) * np.linspace(2.0, 0.2, m)[None, :]).astype(np.float32)
+    Om = gen.projection_signs(rng, m, k)
+    Wd, Omd = torch.from_numpy(W).cuda(), torch.from_numpy(Om).cuda()
+    ws = torch.empty(dbf.load_library().dbf_factorize_workspace_bytes(n, m, k), dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dbf.dbf_factorize_start(Wd, Omd, workspace=ws)  # untimed: the first call creates the cuBLAS handle
+    torch.cuda.synchronize()
+    e0.record()
+    L, R, err = dbf.dbf_factorize_start(Wd, Omd, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    start_ms = e0.elapsed_time(e1)
+    errors, times = [float(err.item())], []
+    for _ in range(args.fact_passes):
+        e0.record()
+        err = dbf.dbf_factorize_pass(Wd, L, R, admm_steps=20, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        errors.append(float(err.item()))
+    steps = 20
+    # GEMMs of one pass: per factor G (k*k*inner), the right-hand product (rows*k*inner), Newton-Schulz 16 x 2 k^3,
+    # per ADMM step one (rows x k x k) product; the error product n*m*k
+    fl = 2.0 * (k * k * m + n * k * m + 32 * k ** 3 + steps * n * k * k) + 2.0 * (k * k * n + k * m * n + 32 * k ** 3 +
+                                                                                  steps * k * m * k) + 2.0 * n * m * k
+    ms = statistics.median(times)
+    print(json.dumps({"factorize": {"n": n, "m": m, "k": k, "bits_per_weight": k * (n + m) / (n * m),
+                                    "start_ms": start_ms, "ms_per_pass": ms, "pass_ms": times,
+                                    "gemm_tflops": fl / (ms * 1e-3) / 1e12, "relative_errors": errors}}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -857,11 +906,16 @@ def main():
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many dbf_forward calls of one layer (for ncu captures)")
     ap.add_argument("--flags", type=int, default=1, help="dbf_forward flags for --profile-calls (default: weights static)")
+    ap.add_argument("--factorize", action="store_true", help="time the offline factorisation of a 4096^2 weight")
+    ap.add_argument("--fact-k", type=int, default=2048)
+    ap.add_argument("--fact-passes", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     shape = gen.CONFIGS[args.workload]
-    if args.profile_calls > 0:
+    if args.factorize:
+        run_factorize(args)
+    elif args.profile_calls > 0:
         run_profile_calls(args, shape, args.batch)
     elif args.sweep:
         run_sweep(args)

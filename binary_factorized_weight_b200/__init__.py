@@ -35,6 +35,8 @@ __all__ = [
     "DBF_MAX_GROUP", "dbf_forward_grouped_workspace_bytes", "dbf_new_grouped_workspace", "dbf_forward_grouped",
     "dbf_transpose_signs", "dbf_forward_transposed",
     "dbf_bqq_prepared_bytes", "dbf_bqq_prepare", "dbf_bqq_workspace_bytes", "dbf_bqq_forward",
+    "dbf_factorize_workspace_bytes", "dbf_factorize_start", "dbf_factorize_pass", "dbf_factorize_finish", "dbf_svid",
+    "dbf_factorize",
 ]
 
 DBF_I8, DBF_F16, DBF_F32 = 0, 1, 2
@@ -69,6 +71,12 @@ EXPORTED_SYMBOLS = (
     "dbf_bqq_prepare",
     "dbf_bqq_workspace_bytes",
     "dbf_bqq_forward",
+    "dbf_factorize_workspace_bytes",
+    "dbf_factorize_start",
+    "dbf_factorize_pass",
+    "dbf_factorize_finish",
+    "dbf_svid_workspace_bytes",
+    "dbf_svid",
     "dbf_status_string",
 )
 
@@ -141,6 +149,18 @@ def load_library():
     lib.dbf_bqq_workspace_bytes.restype = sz
     lib.dbf_bqq_forward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, vp, i32, vp, sz, u32, vp]
     lib.dbf_bqq_forward.restype = i32
+    lib.dbf_factorize_workspace_bytes.argtypes = [i64, i64, i64]
+    lib.dbf_factorize_workspace_bytes.restype = sz
+    lib.dbf_factorize_start.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]
+    lib.dbf_factorize_start.restype = i32
+    lib.dbf_factorize_pass.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp, vp, sz, vp]
+    lib.dbf_factorize_pass.restype = i32
+    lib.dbf_factorize_finish.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dbf_factorize_finish.restype = i32
+    lib.dbf_svid_workspace_bytes.argtypes = [i64, i64]
+    lib.dbf_svid_workspace_bytes.restype = sz
+    lib.dbf_svid.argtypes = [vp, i64, i64, vp, vp, vp, vp, sz, vp]
+    lib.dbf_svid.restype = i32
     lib.dbf_status_string.argtypes = [i32]
     lib.dbf_status_string.restype = ctypes.c_char_p
     _LIB = lib
@@ -385,3 +405,83 @@ def dbf_bqq_forward(x: torch.Tensor, packedY: torch.Tensor, packedZ: torch.Tenso
         _ptr(x), _ptr(packedY), _ptr(packedZ), _ptr(prepared), int(n), int(k), int(p), int(m_in), int(batch),
         _ptr(y), _dtype_code(y.dtype), _ptr(workspace), workspace.numel(), int(flags), _stream(stream)))
     return y
+
+
+def _factorize_ws(n, m, k, device):
+    nbytes = int(load_library().dbf_factorize_workspace_bytes(int(n), int(m), int(k)))
+    if nbytes == 0:
+        raise ValueError("shape outside the factorisation contract")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def dbf_factorize_start(W: torch.Tensor, Omega: torch.Tensor, workspace=None, stream=None):
+    """L = SVID(W Omega), R = SVID(Omega^T); returns (L, R, err) with err a 1-element fp32 CUDA tensor."""
+    n, m = W.shape
+    k = Omega.shape[1]
+    ws = _factorize_ws(n, m, k, W.device) if workspace is None else workspace
+    L = torch.empty((n, k), dtype=torch.float32, device=W.device)
+    R = torch.empty((k, m), dtype=torch.float32, device=W.device)
+    err = torch.empty(4, dtype=torch.float32, device=W.device)
+    _check("dbf_factorize_start", load_library().dbf_factorize_start(
+        _ptr(W), _ptr(Omega), n, m, k, _ptr(L), _ptr(R), _ptr(err), _ptr(ws), ws.numel(), _stream(stream)))
+    return L, R, err[:1]
+
+
+def dbf_factorize_pass(W: torch.Tensor, L: torch.Tensor, R: torch.Tensor, admm_steps: int = 20, workspace=None,
+                       stream=None) -> torch.Tensor:
+    """One alternating pass in place on L (n x k) and R (k x m); returns the error (1-element fp32 CUDA tensor)."""
+    n, m = W.shape
+    k = L.shape[1]
+    ws = _factorize_ws(n, m, k, W.device) if workspace is None else workspace
+    err = torch.empty(4, dtype=torch.float32, device=W.device)
+    _check("dbf_factorize_pass", load_library().dbf_factorize_pass(
+        _ptr(W), n, m, k, _ptr(L), _ptr(R), int(admm_steps), _ptr(err), _ptr(ws), ws.numel(), _stream(stream)))
+    return err[:1]
+
+
+def dbf_factorize_finish(L: torch.Tensor, R: torch.Tensor, workspace=None, stream=None):
+    """The DBF form of an SVID-form pair: (packedA, packedB, a, mid, b)."""
+    n, k = L.shape
+    m = R.shape[1]
+    ws = _factorize_ws(n, m, k, L.device) if workspace is None else workspace
+    pA = torch.empty(dbf_packed_words(n, k), dtype=torch.int32, device=L.device)
+    pB = torch.empty(dbf_packed_words(k, m), dtype=torch.int32, device=L.device)
+    a = torch.empty(n, dtype=torch.float16, device=L.device)
+    mid = torch.empty(k, dtype=torch.float16, device=L.device)
+    b = torch.empty(m, dtype=torch.float16, device=L.device)
+    _check("dbf_factorize_finish", load_library().dbf_factorize_finish(
+        _ptr(L), _ptr(R), n, m, k, _ptr(pA), _ptr(pB), _ptr(a), _ptr(mid), _ptr(b), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return pA, pB, a, mid, b
+
+
+def dbf_svid(M: torch.Tensor, stream=None):
+    """Leading singular pair of |M|: (u, v, sigma) with sign(M) (.) sigma u v^T the SVID projection of M."""
+    rows, cols = M.shape
+    u = torch.empty(rows, dtype=torch.float32, device=M.device)
+    v = torch.empty(cols, dtype=torch.float32, device=M.device)
+    sigma = torch.empty(4, dtype=torch.float32, device=M.device)
+    ws = torch.empty(int(load_library().dbf_svid_workspace_bytes(rows, cols)), dtype=torch.uint8, device=M.device)
+    _check("dbf_svid", load_library().dbf_svid(_ptr(M), rows, cols, _ptr(u), _ptr(v), _ptr(sigma), _ptr(ws),
+                                               ws.numel(), _stream(stream)))
+    return u, v, sigma[:1]
+
+
+def dbf_factorize(W: torch.Tensor, Omega: torch.Tensor, passes: int = 10, admm_steps: int = 20, stream=None):
+    """Factorise a dense fp32 weight (n x m CUDA tensor) with middle dimension k = Omega.shape[1]: the start,
+    `passes` alternating passes keeping the best pair, and the DBF form.  Returns
+    (packedA, packedB, a, mid, b, errors) with errors the relative error of the start and after each pass
+    (non-increasing)."""
+    n, m = W.shape
+    k = Omega.shape[1]
+    ws = _factorize_ws(n, m, k, W.device)
+    L, R, err = dbf_factorize_start(W, Omega, workspace=ws, stream=stream)
+    best = float(err.item())
+    errors = [best]
+    for _ in range(passes):
+        Lc, Rc = L.clone(), R.clone()
+        e = float(dbf_factorize_pass(W, Lc, Rc, admm_steps, workspace=ws, stream=stream).item())
+        if e < best:
+            L, R, best = Lc, Rc, e
+        errors.append(best)
+    return (*dbf_factorize_finish(L, R, workspace=ws, stream=stream), errors)

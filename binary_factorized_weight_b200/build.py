@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdbf.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["dbf_api.cu", "decode.cu", "fused.cu", "prefill.cu", "pack.cu", "transpose.cu", "reconstruct.cu", "bqq.cu", "noalloc.cu"]
+SOURCES = ["dbf_api.cu", "decode.cu", "fused.cu", "prefill.cu", "pack.cu", "transpose.cu", "reconstruct.cu", "bqq.cu", "factorize.cu", "noalloc.cu"]
 HEADERS = ["dbf_device.cuh", "dbf_internal.h"]
 
 NVCC_FLAGS = [
@@ -74,7 +74,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as pool:
         objs = list(pool.map(compile_one, SOURCES))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
+    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs,
+           "-lcublas"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")

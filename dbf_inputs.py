@@ -38,6 +38,7 @@ __all__ = [
     "normal_activations",
     "integer_activations",
     "sylvester_hadamard",
+    "projection_signs",
     "make_layer",
 ]
 
@@ -122,6 +123,12 @@ def normal_activations(rng: np.random.Generator, batch: int, m_in: int) -> np.nd
 def integer_activations(rng: np.random.Generator, batch: int, m_in: int, lo: int = -8, hi: int = 8) -> np.ndarray:
     """Uniform integers in [lo, hi] stored as fp16 (exact), shape (batch, m_in)."""
     return rng.integers(lo, hi + 1, size=(batch, m_in)).astype(np.float16)
+
+
+def projection_signs(rng: np.random.Generator, rows: int, cols: int) -> np.ndarray:
+    """A rows x cols random sign matrix scaled by 1/sqrt(rows), as fp32 (the
+    random projection that starts a factorisation)."""
+    return (sign_matrix(rng, rows, cols).astype(np.float64) / np.sqrt(rows)).astype(np.float32)
 
 
 def sylvester_hadamard(p: int) -> np.ndarray:

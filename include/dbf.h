@@ -352,6 +352,59 @@ DBF_API dbf_status dbf_bqq_forward(const uint16_t* x, const uint32_t* packedY, c
                                    void* y, dbf_dtype y_t, void* workspace, size_t ws_bytes, uint32_t flags,
                                    struct CUstream_st* stream);
 
+/*
+ * Offline factorisation of a dense weight into the DBF form (gist.science
+ * technical summary, section 2.2, optimisation algorithm: alternating
+ * minimisation over the two factors, ADMM for each sign-constrained problem,
+ * SVID projection onto "sign matrix times rank-one magnitudes").  Not a hot
+ * path: it prepares weights once.
+ *
+ * The factors are dense fp32 matrices in SVID form: L = diag(a) A diag(mL)
+ * (n x k) and R = diag(mR) B diag(b) (k x m), W ~= L R.  The caller provides the
+ * starting pair (dbf_factorize_start: a random projection of W's range) and
+ * runs passes, keeping the best pair; dbf_factorize_finish turns it into the
+ * packed signs and fp16 scales that dbf_forward takes.
+ *
+ * dbf_factorize_pass: one alternating pass, in place on L and R:
+ *   left:  G = 2 R R^T + rho I, rho = trace(2 R R^T)/k; Z = L, U = 0;
+ *          admm_steps times: L' = (2 W R^T + rho (Z - U)) G^-1,
+ *          Z = SVID(L' + U), U += L' - Z;  then L = Z;
+ *   right: the same for R with L fixed; then *err = ||W - L R||_F / ||W||_F
+ *   (one fp32 in device memory).  A pass need not lower the error: keep the
+ *   best pair (the Python binding's dbf_factorize does).
+ *   W: n x m fp32 row-major; L: n x k; R: k x m (device, row-major, fp32).
+ *   workspace: dbf_factorize_workspace_bytes(n, m, k) bytes of device memory.
+ *   Shape: n, m <= 65536, k <= 16384, n*m and k*max(n, m) <= 2^31.
+ *   Arithmetic: fp32 (cuBLAS SGEMM for the dense products, no tensor-op math);
+ *   G^-1 by 16 Newton-Schulz steps (G's eigenvalues lie in [rho, rho +
+ *   lambda_max(2 R R^T)], rho their mean); SVID's magnitudes by 30 power
+ *   steps on |M|.  Deterministic.
+ * dbf_svid: the leading singular pair of |M| (rows x cols, fp32): unit vectors
+ *   u (rows) and v (cols) and sigma (one fp32), all device memory (scratch:
+ *   dbf_svid_workspace_bytes(rows, cols) bytes of device workspace), so that
+ *   sign(M) (.) (sigma u v^T) is M's SVID projection (a = sqrt(sigma) u,
+ *   b = sqrt(sigma) v in the DBF scale vectors).
+ */
+/* dbf_factorize_start: L = SVID(W Omega) (n x k), R = SVID(Omega^T) (k x m) for a
+ *   caller-drawn m x k projection Omega (fp32; e.g. random signs / sqrt(m)), and
+ *   *err = the start's relative error.
+ * dbf_factorize_finish: the DBF form of a pair in SVID form: packedA / packedB
+ *   (dbf_packed_words(n, k) / (k, m) words, a set bit where L / R is negative),
+ *   a (n), mid (k), b (m) fp16 with W ~= (a (.) A (.) mid^T)(B (.) b^T). */
+DBF_API size_t dbf_factorize_workspace_bytes(int64_t n, int64_t m, int64_t k);
+DBF_API dbf_status dbf_factorize_start(const float* W, const float* Omega, int64_t n, int64_t m, int64_t k, float* L,
+                                       float* R, float* err, void* workspace, size_t ws_bytes,
+                                       struct CUstream_st* stream);
+DBF_API dbf_status dbf_factorize_finish(const float* L, const float* R, int64_t n, int64_t m, int64_t k,
+                                        uint32_t* packedA, uint32_t* packedB, uint16_t* a, uint16_t* mid, uint16_t* b,
+                                        void* workspace, size_t ws_bytes, struct CUstream_st* stream);
+DBF_API dbf_status dbf_factorize_pass(const float* W, int64_t n, int64_t m, int64_t k, float* L, float* R,
+                                      int admm_steps, float* err, void* workspace, size_t ws_bytes,
+                                      struct CUstream_st* stream);
+DBF_API size_t dbf_svid_workspace_bytes(int64_t rows, int64_t cols);
+DBF_API dbf_status dbf_svid(const float* M, int64_t rows, int64_t cols, float* u, float* v, float* sigma,
+                            void* workspace, size_t ws_bytes, struct CUstream_st* stream);
+
 /* Static, NUL-terminated description of a status code. */
 DBF_API const char* dbf_status_string(dbf_status status);
 
