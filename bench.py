@@ -429,7 +429,10 @@ def roofline_for(wl, shape, batch, us, peaks, traffic, peak_kind="burst"):
 
 def measure_workload(dbf, torch, shape, batch, device, peaks, rounds=5):
     """One more configuration of the metric in the same run: R rotated copies in
-    one CUDA graph, device-timed; its own roofline."""
+    one CUDA graph, device-timed; its own roofline and clock record.  A
+    tensor-core configuration whose timed rounds run back to back for 100 ms or
+    more is a kernel timed inside a long step: its fraction is taken of the
+    sustained dense peak (the burst fraction is given beside it)."""
     wl = Workload(dbf, torch, shape, batch, device)
     g = wl.capture()
     launches = graph_kernel_launches(g)
@@ -437,15 +440,26 @@ def measure_workload(dbf, torch, shape, batch, device, peaks, rounds=5):
         g.replay()
     torch.cuda.synchronize()
     reps = max(3, int(400 / wl.copies))
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)  # nvidia-smi's first samples (outside the timed region)
+    t0 = time.time()
     ms = time_replays(torch, g, reps, rounds)
+    t1 = time.time()
+    sampler.stop()
     us = 1e3 * ms / reps / wl.copies
     ok = dbf.dbf_workspace_status(wl.ws) == 0
+    long_run = (t1 - t0) >= 0.1
+    roof = roofline_for(wl, shape, batch, us, peaks, traffic_for(f"{shape.name}_b{batch}"),
+                        peak_kind="sustained" if (batch > 16 and long_run) else "burst")
+    if batch > 16:
+        roof["frac_of_burst"] = roof["achieved"] / peaks["bf16_tflops"]
+        roof["timed_seconds"] = round(t1 - t0, 3)
     out = {"workload": workload_name(shape, batch), "path": path_name(wl, None if launches is None else
                                                                          launches / wl.copies),
            "us_per_layer": us, "tokens_per_s": batch / (us * 1e-6), "layers_per_replay": wl.copies,
            "launches_per_layer": None if launches is None else launches / wl.copies,
-           "roofline": roofline_for(wl, shape, batch, us, peaks, traffic_for(f"{shape.name}_b{batch}")),
-           "status_ok": ok}
+           "roofline": roof, "clocks": sampler.summary(t0, t1), "status_ok": ok}
     del g, wl
     torch.cuda.empty_cache()
     return out

@@ -67,18 +67,27 @@ constexpr int kWarpEpi0 = kWarpMma + 1;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kEpiStageBytes = 32 * 32 * 4;  // one warp's 32 tokens x 32 rows (fp32 worst case)
 
-template <int NTILE, bool SPLIT>
+template <int NTILE, bool SPLIT, bool ATMEM>
 struct Cfg {
-  static constexpr int kStages = NTILE == 256 ? 4 : 6;
+  // TMEM accumulators: two, so that the epilogue of one tile overlaps the
+  // main loop of the next, except for 256-token tiles with A in TMEM, where
+  // the A ring takes the room of the second one
+  static constexpr int kAccBufs = (ATMEM && NTILE == 256) ? 1 : 2;
+  static constexpr int kStages = ATMEM ? (NTILE == 256 ? 4 : 8) : (NTILE == 256 ? 4 : 6);
+  static constexpr int kAStageBytes = ATMEM ? 0 : kABytes;  // A in TMEM: no shared-memory A ring
   static constexpr int kBBytes = NTILE * kBK * 2;
-  static constexpr int kEpiOffset = kStages * (kABytes + kBBytes);
+  static constexpr int kEpiOffset = kStages * (kAStageBytes + kBBytes);
   static constexpr int kBarOffset = kEpiOffset + 4 * kEpiStageBytes;
   // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done, recv
   static constexpr int kNumBars = 3 * kStages + 6;
   static constexpr int kRsOffset = kBarOffset + kNumBars * 8 + 16;  // after the tmem slot and abort flag
   // + split K: the tile's row scales (fp32), + alignment slack
   static constexpr int kSmemBytes = kRsOffset + kBM * 4 + 1024;
-  static constexpr int kTmemCols = 2 * NTILE;
+  // TMEM: kAccBufs accumulators of NTILE columns, then (A in TMEM) the A
+  // ring, kBK / 2 columns per stage (column c of a stage = the fp16 pair K 2c, 2c+1)
+  static constexpr int kTmemA = kAccBufs * NTILE;
+  static constexpr int kTmemCols = ATMEM ? 512 : 2 * NTILE;
+  static_assert(!ATMEM || kTmemA + kStages * (kBK / 2) <= 512, "A ring must fit in tensor memory");
   // split K: once a CTA's MMAs are done its operand rings are idle; the B ring
   // then receives the peers' parts of this CTA's token columns,
   // [src rank][NTILE/ks/4][128 rows] float4 (at most one whole partial tile).
@@ -87,15 +96,15 @@ struct Cfg {
   static_assert(!SPLIT || 14 * 8 * 32 * 4 <= 4 * kEpiStageBytes, "split-K output transposes must fit the epilogue stage");
 };
 
-template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32>
+template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32, bool ATMEM>
 __global__ void __launch_bounds__(kThreads, 1)
     dbf_prefill_gemm_kernel(const __grid_constant__ CUtensorMap act_map, const PrefillArgs p) {
-  using C = Cfg<NTILE, SPLIT>;
+  using C = Cfg<NTILE, SPLIT, ATMEM>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_st = smem;
-  uint8_t* b_st = smem + S * kABytes;
+  uint8_t* b_st = smem + S * C::kAStageBytes;
   uint8_t* epi_st = smem + C::kEpiOffset;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* full_a = bars;
@@ -160,10 +169,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ sign expansion
     // Row r's packed row is a sequence of 8-word blocks of 256 columns; K step
     // kt covers groups 4*(kt%4) .. 4*(kt%4)+3 of block kt/4, and group g's 16
-    // columns come from bit pair (g, g+16) of the block's 8 words.  This thread
-    // holds words 4h..4h+3 (column pairs 4h..4h+3 of every group).
+    // columns come from bit pair (g, g+16) of the block's 8 words.
+    // A in shared memory: thread (row, h) holds words 4h..4h+3 (column pairs
+    // 4h..4h+3 of every group) and writes four 16-byte chunks per K step.
+    // A in tensor memory: thread (row, h) holds all 8 words and writes the 16
+    // column pairs of groups 2h, 2h+1 of each K step (TMEM columns 16h..16h+15
+    // of the stage, one 32x32b.x16 store per warp into its TMEM lane quadrant).
     const int r_local = tid & (kBM - 1);
     const int h = tid >> 7;
+    struct Words {
+      uint4 lo, hi;  // hi: words 4..7 (A in tensor memory only)
+    };
     // block sequence of this CTA: (item, blk) with blk fastest
     int f_w = blockIdx.x, f_blk = 0, f_end = 0;
     auto f_seek = [&]() {
@@ -174,11 +190,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     f_seek();
-    auto fetch_next = [&]() -> uint4 {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    auto fetch_next = [&]() -> Words {
+      Words v{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
       if (f_w < num_items) {
         const int r = ((f_w / ks) % m_tiles) * kBM + r_local;
-        if (r < p.M) v = ldg_stream_u4(p.packed + static_cast<int64_t>(r) * p.wpr + 8 * f_blk + 4 * h);
+        if (r < p.M) {
+          const uint32_t* src = p.packed + static_cast<int64_t>(r) * p.wpr + 8 * f_blk;
+          if constexpr (ATMEM) {
+            v.lo = ldg_stream_u4(src);
+            v.hi = ldg_stream_u4(src + 4);
+          } else {
+            v.lo = ldg_stream_u4(src + 4 * h);
+          }
+        }
         if (++f_blk == f_end) {
           f_w += gridDim.x;
           f_seek();
@@ -186,15 +210,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return v;
     };
+    // The scale pairs of this thread's columns of K step kt: A in shared
+    // memory, sc[i] = columns 16i + 8h .. +7; A in tensor memory,
+    // sc[2j + c] = columns 16(2h + j) + 8c .. +7.
     auto fetch_scale = [&](int kt, uint4 (&sc)[4]) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        sc[i] = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + 16 * i + 8 * h));
+      for (int i = 0; i < 4; ++i) {
+        const int col = ATMEM ? 16 * (2 * h + (i >> 1)) + 8 * (i & 1) : 16 * i + 8 * h;
+        sc[i] = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + col));
+      }
     };
     int first_b0 = 0, first_b1 = 0;
     if (static_cast<int>(blockIdx.x) < num_items) item_blocks(blockIdx.x, first_b0, first_b1);
     const int kt_first = min(KT - 1, 4 * first_b0);
-    uint4 w_n1, w_n2, wcur = make_uint4(0u, 0u, 0u, 0u);
+    Words w_n1, w_n2, wcur{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
     uint4 sc_next[4];
     if (p.weights_early) {
       w_n1 = fetch_next();
@@ -209,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bool ok = true;
     const int swz = r_local & 7;
+    const uint32_t a_lane = static_cast<uint32_t>(r_local & ~31) << 16;  // this warp's TMEM lane quadrant
     uint32_t it = 0;
     for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
       int b0, b1;
@@ -222,37 +252,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           w_n1 = w_n2;
           w_n2 = fetch_next();
         }
+        // the next K step (the next item of a persistent CTA starts again at K step 0)
+        const int kt_next = kt + 1 < kt1 ? kt + 1 : (SPLIT ? kt0 : 0);
         uint4 sc[4];
         if constexpr (KSCALE) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) sc[i] = sc_next[i];
-          // the next item of a persistent CTA starts again at K step 0
-          fetch_scale(kt + 1 < kt1 ? kt + 1 : (SPLIT ? kt0 : 0), sc_next);
+          fetch_scale(kt_next, sc_next);
         }
         if (it >= S && !mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
-        uint8_t* dst = a_st + s * kABytes + (r_local >> 3) * 1024 + swz * 128;
+        if constexpr (ATMEM) {
+          tc_fence_after();  // the MMAs that read this stage have completed
+          const uint32_t wd[8] = {wcur.lo.x, wcur.lo.y, wcur.lo.z, wcur.lo.w, wcur.hi.x, wcur.hi.y, wcur.hi.z, wcur.hi.w};
+          uint32_t q[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int g = 4 * (kt & 3) + i;  // group inside the block
-          uint32_t q[4];
-          if constexpr (KSCALE) {
-            q[0] = signed_scale_pair_rt(wcur.x, g, sc[i].x);
-            q[1] = signed_scale_pair_rt(wcur.y, g, sc[i].y);
-            q[2] = signed_scale_pair_rt(wcur.z, g, sc[i].z);
-            q[3] = signed_scale_pair_rt(wcur.w, g, sc[i].w);
-          } else {
-            q[0] = pm1_pair_rt(wcur.x, g);
-            q[1] = pm1_pair_rt(wcur.y, g);
-            q[2] = pm1_pair_rt(wcur.z, g);
-            q[3] = pm1_pair_rt(wcur.w, g);
+          for (int j = 0; j < 2; ++j) {
+            const int g = 4 * (kt & 3) + 2 * h + j;  // group inside the block
+#pragma unroll
+            for (int pr = 0; pr < 8; ++pr) {
+              if constexpr (KSCALE) {
+                const uint4 v = sc[2 * j + (pr >> 2)];
+                const uint32_t sp = (pr & 3) == 0 ? v.x : (pr & 3) == 1 ? v.y : (pr & 3) == 2 ? v.z : v.w;
+                q[8 * j + pr] = signed_scale_pair_rt(wd[pr], g, sp);
+              } else {
+                q[8 * j + pr] = pm1_pair_rt(wd[pr], g);
+              }
+            }
           }
-          // columns 16i + 8h .. 16i + 8h + 7 -> 16-byte chunk 2i + h (128B swizzle)
-          *reinterpret_cast<uint4*>(dst + (((2 * i + h) ^ swz) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+          tmem_st_32x32b_x16(tmem_base + a_lane + static_cast<uint32_t>(C::kTmemA + s * (kBK / 2) + 16 * h), q);
+          tmem_st_wait();
+          tc_fence_before();
+        } else {
+          uint8_t* dst = a_st + s * kABytes + (r_local >> 3) * 1024 + swz * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int g = 4 * (kt & 3) + i;  // group inside the block
+            uint32_t q[4];
+            if constexpr (KSCALE) {
+              q[0] = signed_scale_pair_rt(wcur.lo.x, g, sc[i].x);
+              q[1] = signed_scale_pair_rt(wcur.lo.y, g, sc[i].y);
+              q[2] = signed_scale_pair_rt(wcur.lo.z, g, sc[i].z);
+              q[3] = signed_scale_pair_rt(wcur.lo.w, g, sc[i].w);
+            } else {
+              q[0] = pm1_pair_rt(wcur.lo.x, g);
+              q[1] = pm1_pair_rt(wcur.lo.y, g);
+              q[2] = pm1_pair_rt(wcur.lo.z, g);
+              q[3] = pm1_pair_rt(wcur.lo.w, g);
+            }
+            // columns 16i + 8h .. 16i + 8h + 7 -> 16-byte chunk 2i + h (128B swizzle)
+            *reinterpret_cast<uint4*>(dst + (((2 * i + h) ^ swz) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         mbar_arrive(&full_a[s]);
       }
     }
@@ -286,8 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       uint32_t it = 0, local = 0;
       for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x, ++local) {
-        const uint32_t buf = local & 1;
-        if (local >= 2 && !mbar_wait_bounded(&acc_empty[buf], ((local >> 1) - 1) & 1, abort_flag, p.status)) {
+        const uint32_t buf = local % C::kAccBufs;
+        if (local >= C::kAccBufs &&
+            !mbar_wait_bounded(&acc_empty[buf], ((local / C::kAccBufs) - 1) & 1, abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -305,12 +360,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(a_st + s * kABytes);
+          const uint32_t a_addr = smem_u32(a_st + s * C::kAStageBytes);
           const uint32_t b_addr = smem_u32(b_st + s * C::kBBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            tc_mma_f16_ss(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32), smem_desc_sw128_kmajor(b_addr + kk * 32),
-                          idesc, (kt != kt0 || kk != 0) ? 1u : 0u);
+            const uint32_t acc = (kt != kt0 || kk != 0) ? 1u : 0u;
+            if constexpr (ATMEM) {
+              tc_mma_f16_ts(d_tmem, tmem_base + static_cast<uint32_t>(C::kTmemA + s * (kBK / 2) + kk * 8),
+                            smem_desc_sw128_kmajor(b_addr + kk * 32), idesc, acc);
+            } else {
+              tc_mma_f16_ss(d_tmem, smem_desc_sw128_kmajor(a_addr + kk * 32), smem_desc_sw128_kmajor(b_addr + kk * 32),
+                            idesc, acc);
+            }
           }
           tc_commit(&empty[s]);
         }
@@ -336,13 +397,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
       const bool ld_ok = (p.ld_out % kVec) == 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-        const uint32_t buf = local & 1;
+        const uint32_t buf = local % C::kAccBufs;
         const int m0 = (tile % m_tiles) * kBM;
         const int n0 = (tile / m_tiles) * NTILE;
         const int row0 = m0 + q * 32;
         const int row = row0 + lane;
         const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;  // in flight during the wait
-        if (!mbar_wait_bounded(&acc_full[buf], (local >> 1) & 1, abort_flag, p.status)) break;
+        if (!mbar_wait_bounded(&acc_full[buf], (local / C::kAccBufs) & 1, abort_flag, p.status)) break;
         tc_fence_after();
         const bool rows_full = row0 + 32 <= p.M;
         for (int col = 0; col < NTILE; col += 32) {
@@ -557,11 +618,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32>
+template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32, bool ATMEM>
 dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, const DeviceInfo& dev,
                         cudaStream_t stream) {
-  auto kernel = dbf_prefill_gemm_kernel<NTILE, SPLIT, KSCALE, OUT_F32>;
-  constexpr int smem = Cfg<NTILE, SPLIT>::kSmemBytes;
+  auto kernel = dbf_prefill_gemm_kernel<NTILE, SPLIT, KSCALE, OUT_F32, ATMEM>;
+  constexpr int smem = Cfg<NTILE, SPLIT, ATMEM>::kSmemBytes;
   static std::once_flag once;  // the attribute once per instantiation
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] { attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); });
@@ -587,14 +648,14 @@ dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, co
   return cudaLaunchKernelEx(&cfg, kernel, map, a) == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
-template <int NTILE, bool SPLIT>
+template <int NTILE, bool SPLIT, bool ATMEM>
 dbf_status launch_split(const PrefillArgs& a, const CUtensorMap& map, int ks, bool out_f32, const DeviceInfo& dev,
                         cudaStream_t stream) {
   if (a.kscale != nullptr)
-    return out_f32 ? launch_typed<NTILE, SPLIT, true, true>(a, map, ks, dev, stream)
-                   : launch_typed<NTILE, SPLIT, true, false>(a, map, ks, dev, stream);
-  return out_f32 ? launch_typed<NTILE, SPLIT, false, true>(a, map, ks, dev, stream)
-                 : launch_typed<NTILE, SPLIT, false, false>(a, map, ks, dev, stream);
+    return out_f32 ? launch_typed<NTILE, SPLIT, true, true, ATMEM>(a, map, ks, dev, stream)
+                   : launch_typed<NTILE, SPLIT, true, false, ATMEM>(a, map, ks, dev, stream);
+  return out_f32 ? launch_typed<NTILE, SPLIT, false, true, ATMEM>(a, map, ks, dev, stream)
+                 : launch_typed<NTILE, SPLIT, false, false, ATMEM>(a, map, ks, dev, stream);
 }
 
 }  // namespace
@@ -663,8 +724,8 @@ static int max_resident_clusters(int device, int ks, int num_sms) {
   const auto key = std::make_pair(device, ks);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  auto kernel = dbf_prefill_gemm_kernel<128, true, false, false>;
-  constexpr int smem = Cfg<128, true>::kSmemBytes;
+  auto kernel = dbf_prefill_gemm_kernel<128, true, false, false, true>;
+  constexpr int smem = Cfg<128, true, true>::kSmemBytes;
   int n = 0;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -735,9 +796,13 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
   CUtensorMap map;
   if (!activation_map(act, a.K, act_rows, ntile, encode, &map)) return DBF_ERR_CUDA;
 
-  if (ks > 1) return launch_split<128, true>(a, map, ks, out_f32, dev, stream);
-  if (ntile == 256) return launch_split<256, false>(a, map, 1, out_f32, dev, stream);
-  return launch_split<128, false>(a, map, 1, out_f32, dev, stream);
+  if (ks > 1) return launch_split<128, true, true>(a, map, ks, out_f32, dev, stream);
+  // 256-token tiles keep A in shared memory for fp32 outputs (the single
+  // accumulator's drain would take twice as long)
+  if (ntile == 256)
+    return out_f32 ? launch_split<256, false, false>(a, map, 1, true, dev, stream)
+                   : launch_split<256, false, true>(a, map, 1, false, dev, stream);
+  return launch_split<128, false, true>(a, map, 1, out_f32, dev, stream);
 }
 
 }  // namespace dbf
