@@ -89,22 +89,30 @@ dbf_status dbf_pack_signs(const void* src, dbf_dtype src_t, int64_t rows, int64_
 
 namespace {
 // Workspace layout: status block, V (batch x k fp16, the two-launch and
-// tensor-core paths), then the tagged partials of the single-launch decode
-// (batch x n x 8 64-bit words; only for batch <= 16).
+// tensor-core paths), then either the tagged partials of the single-launch
+// decode (batch x n x 8 64-bit words; batch <= 16) or the stream-K flags and
+// partial-tile slots of the tensor-core path (batch > 128).  The last area is
+// optional: with less room the forward runs a schedule that does not use it.
 size_t v_area_end(int64_t k, int64_t batch) {
   const size_t v_bytes = static_cast<size_t>(batch) * static_cast<size_t>(k) * 2;
   return kStatusBytes + (v_bytes + 255) / 256 * 256;
 }
+size_t sk_area_bytes(int64_t batch) { return batch > 128 ? kSkBytes : 0; }
 size_t slot_bytes(int64_t n, int64_t tokens) {
   return static_cast<size_t>(kFusedMaxSlices) * static_cast<size_t>(tokens) * static_cast<size_t>(n) * 8;
 }
 }  // namespace
 
+size_t dbf::forward_workspace_min_bytes(int64_t k, int64_t batch) {
+  if (k < 1 || batch < 1) return 0;
+  return v_area_end(k, batch);
+}
+
 extern "C" {
 
 size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, int64_t batch) {
   if (n < 1 || k < 1 || m_in < 1 || batch < 1) return 0;
-  return v_area_end(k, batch) + (batch <= 16 ? slot_bytes(n, batch) : 0);
+  return v_area_end(k, batch) + (batch <= 16 ? slot_bytes(n, batch) : 0) + sk_area_bytes(batch);
 }
 
 static dbf_status validate_factors(const uint32_t* packedA, const uint32_t* packedB, const uint16_t* a,
@@ -150,8 +158,7 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
                        struct CUstream_st* stream_handle) {
   dbf_status st = validate_forward_args(x, packedA, packedB, a, m, b, n, k, m_in, batch, y, y_t, flags);
   if (st != DBF_OK) return st;
-  if (!workspace || !aligned16(workspace) || ws_bytes < dbf_forward_workspace_bytes(n, k, m_in, batch))
-    return DBF_ERR_WORKSPACE;
+  if (!workspace || !aligned16(workspace) || ws_bytes < v_area_end(k, batch)) return DBF_ERR_WORKSPACE;
   DeviceInfo dev;
   st = current_device(&dev);
   if (st != DBF_OK) return st;
@@ -238,7 +245,12 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
     return DBF_OK;
   }
 
+  // stream-K scratch after V, when the workspace has room for it
+  char* sk = ws_bytes >= v_area_end(k, batch) + kSkBytes ? static_cast<char*>(workspace) + v_area_end(k, batch)
+                                                         : nullptr;
   PrefillArgs g1{};
+  g1.sk_flags = sk ? reinterpret_cast<unsigned*>(sk) : nullptr;
+  g1.sk_slots = sk ? reinterpret_cast<float*>(sk + kSkFlagBytes) : nullptr;
   g1.packed = packedB;
   g1.wpr = words_per_row(m_in);
   g1.M = static_cast<int>(k);
@@ -253,6 +265,8 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
   st = launch_prefill_gemm(g1, xh, batch, /*out_f32=*/false, dev, stream);
   if (st != DBF_OK) return st;
   PrefillArgs g2{};
+  g2.sk_flags = g1.sk_flags;
+  g2.sk_slots = g1.sk_slots;
   g2.packed = packedA;
   g2.wpr = words_per_row(k);
   g2.M = static_cast<int>(n);
@@ -278,7 +292,7 @@ size_t dbf_forward_grouped_workspace_bytes(const dbf_layer_desc* layers, int num
   if (!layers || num_layers < 1 || num_layers > DBF_MAX_GROUP || m_in < 1 || batch < 1) return 0;
   for (int g = 0; g < num_layers; ++g)
     if (layers[g].n < 1 || layers[g].k < 1) return 0;
-  return grouped_v_offset(layers, num_layers, batch);
+  return grouped_v_offset(layers, num_layers, batch) + sk_area_bytes(batch);
 }
 
 dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, const dbf_layer_desc* layers,
@@ -302,8 +316,7 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
   if ((flags & ~known) != 0) return DBF_ERR_INVALID_ARG;
   if ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)) return DBF_ERR_INVALID_ARG;
   if (!aligned16(x)) return DBF_ERR_MISALIGNED;
-  if (!workspace || !aligned16(workspace) ||
-      ws_bytes < dbf_forward_grouped_workspace_bytes(layers, num_layers, m_in, batch))
+  if (!workspace || !aligned16(workspace) || ws_bytes < grouped_v_offset(layers, num_layers, batch))
     return DBF_ERR_WORKSPACE;
   DeviceInfo dev;
   dbf_status st = current_device(&dev);
@@ -373,7 +386,11 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
   // Large batches are tensor-core bound: one layer after the other.
   for (int g = 0; g < num_layers; ++g) {
     const dbf_layer_desc& l = layers[g];
+    const size_t v_end = grouped_v_offset(layers, num_layers, batch);
+    char* sk = ws_bytes >= v_end + kSkBytes ? static_cast<char*>(workspace) + v_end : nullptr;
     PrefillArgs g1{};
+    g1.sk_flags = sk ? reinterpret_cast<unsigned*>(sk) : nullptr;
+    g1.sk_slots = sk ? reinterpret_cast<float*>(sk + kSkFlagBytes) : nullptr;
     g1.packed = l.packedB;
     g1.wpr = words_per_row(m_in);
     g1.M = static_cast<int>(l.k);
@@ -388,6 +405,8 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
     st = launch_prefill_gemm(g1, xh, batch, /*out_f32=*/false, dev, stream);
     if (st != DBF_OK) return st;
     PrefillArgs g2{};
+    g2.sk_flags = g1.sk_flags;
+    g2.sk_slots = g1.sk_slots;
     g2.packed = l.packedA;
     g2.wpr = words_per_row(l.k);
     g2.M = static_cast<int>(l.n);

@@ -43,7 +43,17 @@ struct PrefillArgs {
   int batch;
   int weights_early;
   int* status;  // device status word (DBF_ERR_TIMEOUT on a lost wait)
+  // stream-K scratch (null: no stream-K schedule): kSkMaxCtas partial tiles of
+  // 128 x 256 fp32 and kSkMaxCtas flags, zero between launches
+  float* sk_slots;
+  unsigned* sk_flags;
 };
+
+// Stream-K: at most this many CTAs, one partial tile slot each.
+constexpr int kSkMaxCtas = 160;
+constexpr size_t kSkFlagBytes = 1024;  // kSkMaxCtas 32-bit flags, padded
+constexpr size_t kSkSlotBytes = size_t{128} * 256 * 4;
+constexpr size_t kSkBytes = kSkFlagBytes + kSkMaxCtas * kSkSlotBytes;
 
 struct DeviceInfo {
   int device;
@@ -52,6 +62,10 @@ struct DeviceInfo {
 };
 
 dbf_status current_device(DeviceInfo* info);
+
+// The smallest workspace dbf_forward accepts (status block and V); the
+// optional areas after it enable the single-launch decode and stream-K.
+size_t forward_workspace_min_bytes(int64_t k, int64_t batch);
 
 // The synchronous argument checks of dbf_forward other than the workspace
 // (shared by every entry point that runs the layer forward).

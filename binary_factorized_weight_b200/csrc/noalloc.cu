@@ -61,7 +61,9 @@ dbf_status dbf_forward_noalloc(const uint16_t* x, const uint32_t* packedA, const
                                struct CUstream_st* stream) {
   dbf_status st = dbf::validate_forward_args(x, packedA, packedB, a, m, b, n, k, m_in, batch, y, y_t, flags);
   if (st != DBF_OK) return st;
-  if (dbf_forward_workspace_bytes(n, k, m_in, batch) > kNoAllocScratchBytes) return DBF_ERR_WORKSPACE;
+  // the buffer holds the status block and V; the optional areas after them
+  // (single-launch decode partials, stream-K slots) are used where they fit
+  if (dbf::forward_workspace_min_bytes(k, batch) > kNoAllocScratchBytes) return DBF_ERR_WORKSPACE;
   dbf::DeviceInfo dev;
   st = dbf::current_device(&dev);
   if (st != DBF_OK) return st;

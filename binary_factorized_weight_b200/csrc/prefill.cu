@@ -67,6 +67,32 @@ constexpr int kWarpEpi0 = kWarpMma + 1;
 constexpr int kABytes = kBM * kBK * 2;
 constexpr int kEpiStageBytes = 32 * 32 * 4;  // one warp's 32 tokens x 32 rows (fp32 worst case)
 
+__device__ __forceinline__ void st_release_gpu_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait for a stream-K flag raised by another CTA of this grid (the
+// same budget and abort protocol as the barrier waits).
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned* f, volatile int* abort_flag, int* status) {
+  if (ld_acquire_gpu_u32(f) != 0u) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_gpu_u32(f) != 0u) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+        *abort_flag = 1;
+        if (status) atomicCAS(status, 0, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 template <int NTILE, bool SPLIT, bool ATMEM>
 struct Cfg {
   // TMEM accumulators: two, so that the epilogue of one tile overlaps the
@@ -78,8 +104,8 @@ struct Cfg {
   static constexpr int kBBytes = NTILE * kBK * 2;
   static constexpr int kEpiOffset = kStages * (kAStageBytes + kBBytes);
   static constexpr int kBarOffset = kEpiOffset + 4 * kEpiStageBytes;
-  // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done, recv
-  static constexpr int kNumBars = 3 * kStages + 6;
+  // full_a[S], full_b[S], empty[S], acc_full[2], acc_empty[2], mma_done, recv, epi, sk
+  static constexpr int kNumBars = 3 * kStages + 8;
   static constexpr int kRsOffset = kBarOffset + kNumBars * 8 + 16;  // after the tmem slot and abort flag
   // + split K: the tile's row scales (fp32), + alignment slack
   static constexpr int kSmemBytes = kRsOffset + kBM * 4 + 1024;
@@ -96,9 +122,11 @@ struct Cfg {
   static_assert(!SPLIT || 14 * 8 * 32 * 4 <= 4 * kEpiStageBytes, "split-K output transposes must fit the epilogue stage");
 };
 
-template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32, bool ATMEM>
+template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32, bool ATMEM, bool SK>
 __global__ void __launch_bounds__(kThreads, 1)
     dbf_prefill_gemm_kernel(const __grid_constant__ CUtensorMap act_map, const PrefillArgs p) {
+  static_assert(!(SK && SPLIT), "stream-K and the cluster split are separate schedules");
+  static_assert(!SK || NTILE * kBM * 4 <= static_cast<int>(kSkSlotBytes), "a partial tile must fit its slot");
   using C = Cfg<NTILE, SPLIT, ATMEM>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -114,6 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = bars + 3 * S + 2;
   uint64_t* mma_done = bars + 3 * S + 4;
   uint64_t* recv_bar = bars + 3 * S + 5;  // split K: the peers' parts have landed
+  uint64_t* epi_bar = bars + 3 * S + 6;   // stream-K: the four epilogue warps meet (bounded, unlike bar.sync)
+  uint64_t* sk_bar = bars + 3 * S + 7;    // stream-K: a partial tile has been copied into the B ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* rs_s = reinterpret_cast<float*>(smem + C::kRsOffset);  // split K: row scales of the tile
@@ -136,6 +166,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     b0 = min(nblk, (w % ks) * bper);
     b1 = min(nblk, b0 + bper);
   };
+  // Stream-K: the units (tile, 256-column block), tile-major, are cut into
+  // gridDim.x contiguous ranges, one per CTA; a CTA's range is a sequence of
+  // segments (tile, blocks b0..b1).  Only a CTA's first segment can start
+  // inside a tile (it then leaves an fp32 partial tile in its slot) and only
+  // its last can stop inside one (it then finishes that tile: it adds the
+  // partials of the CTAs after it whose first segments lie in the tile).
+  const int64_t sk_units = static_cast<int64_t>(num_tiles) * nblk;
+  auto sk_lo = [&](int64_t c) { return sk_units * c / gridDim.x; };
+  const int64_t sk_hi = SK ? sk_lo(blockIdx.x + 1) : 0;
+  // A work cursor walks this CTA's work: an item index (one item per tile and
+  // K slice, stepping by gridDim.x) or, for stream-K, a unit index.
+  const int64_t work_first = SK ? sk_lo(blockIdx.x) : static_cast<int64_t>(blockIdx.x);
+  auto work_valid = [&](int64_t c) { return SK ? c < sk_hi : c < num_items; };
+  auto work_get = [&](int64_t c, int& tile, int& b0, int& b1) {
+    if constexpr (SK) {
+      tile = static_cast<int>(c / nblk);
+      b0 = static_cast<int>(c % nblk);
+      const int64_t end = b0 + (sk_hi - c);
+      b1 = end < nblk ? static_cast<int>(end) : nblk;
+    } else {
+      tile = static_cast<int>(c) / ks;
+      item_blocks(static_cast<int>(c), b0, b1);
+    }
+  };
+  auto work_next = [&](int64_t c, int b0, int b1) -> int64_t {
+    return SK ? c + (b1 - b0) : c + static_cast<int64_t>(gridDim.x);
+  };
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
@@ -149,6 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(recv_bar, 1);
+    mbar_init(epi_bar, 128);
+    mbar_init(sk_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -180,20 +239,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     struct Words {
       uint4 lo, hi;  // hi: words 4..7 (A in tensor memory only)
     };
-    // block sequence of this CTA: (item, blk) with blk fastest
-    int f_w = blockIdx.x, f_blk = 0, f_end = 0;
+    // block sequence of this CTA: (work, blk) with blk fastest
+    int64_t f_cur = work_first;
+    int f_tile = 0, f_b0 = 0, f_blk = 0, f_end = 0;
     auto f_seek = [&]() {
-      while (f_w < num_items) {
-        item_blocks(f_w, f_blk, f_end);
+      while (work_valid(f_cur)) {
+        work_get(f_cur, f_tile, f_b0, f_end);
+        f_blk = f_b0;
         if (f_blk < f_end) return;
-        f_w += gridDim.x;
+        f_cur = work_next(f_cur, f_b0, f_end);
       }
     };
     f_seek();
     auto fetch_next = [&]() -> Words {
       Words v{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-      if (f_w < num_items) {
-        const int r = ((f_w / ks) % m_tiles) * kBM + r_local;
+      if (work_valid(f_cur)) {
+        const int r = (f_tile % m_tiles) * kBM + r_local;
         if (r < p.M) {
           const uint32_t* src = p.packed + static_cast<int64_t>(r) * p.wpr + 8 * f_blk;
           if constexpr (ATMEM) {
@@ -204,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (++f_blk == f_end) {
-          f_w += gridDim.x;
+          f_cur = work_next(f_cur, f_b0, f_end);
           f_seek();
         }
       }
@@ -220,8 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         sc[i] = __ldg(reinterpret_cast<const uint4*>(p.kscale + kt * kBK + col));
       }
     };
-    int first_b0 = 0, first_b1 = 0;
-    if (static_cast<int>(blockIdx.x) < num_items) item_blocks(blockIdx.x, first_b0, first_b1);
+    int first_tile = 0, first_b0 = 0, first_b1 = 0;
+    if (work_valid(work_first)) work_get(work_first, first_tile, first_b0, first_b1);
     const int kt_first = min(KT - 1, 4 * first_b0);
     Words w_n1, w_n2, wcur{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
     uint4 sc_next[4];
@@ -240,9 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int swz = r_local & 7;
     const uint32_t a_lane = static_cast<uint32_t>(r_local & ~31) << 16;  // this warp's TMEM lane quadrant
     uint32_t it = 0;
-    for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
-      int b0, b1;
-      item_blocks(w, b0, b1);
+    for (int64_t wc = work_first; work_valid(wc) && ok;) {
+      int tile, b0, b1;
+      work_get(wc, tile, b0, b1);
+      wc = work_next(wc, b0, b1);
       const int kt0 = 4 * b0, kt1 = min(KT, 4 * b1);
       for (int kt = kt0; kt < kt1; ++kt, ++it) {
         const int s = static_cast<int>(it % S);
@@ -316,10 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       pdl_wait();
       uint32_t it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x) {
-        int b0, b1;
-        item_blocks(w, b0, b1);
-        const int n0 = ((w / ks) / m_tiles) * NTILE;
+      for (int64_t wc = work_first; work_valid(wc) && ok;) {
+        int tile, b0, b1;
+        work_get(wc, tile, b0, b1);
+        wc = work_next(wc, b0, b1);
+        const int n0 = (tile / m_tiles) * NTILE;
         for (int kt = 4 * b0; kt < min(KT, 4 * b1); ++kt, ++it) {
           const int s = static_cast<int>(it % S);
           const uint32_t use = it / S;
@@ -339,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_f16_f32(kBM, NTILE);
       bool ok = true;
       uint32_t it = 0, local = 0;
-      for (int w = blockIdx.x; w < num_items && ok; w += gridDim.x, ++local) {
+      for (int64_t wc = work_first; work_valid(wc) && ok; ++local) {
         const uint32_t buf = local % C::kAccBufs;
         if (local >= C::kAccBufs &&
             !mbar_wait_bounded(&acc_empty[buf], ((local / C::kAccBufs) - 1) & 1, abort_flag, p.status)) {
@@ -348,8 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * NTILE;
-        int b0, b1;
-        item_blocks(w, b0, b1);
+        int tile, b0, b1;
+        work_get(wc, tile, b0, b1);
+        wc = work_next(wc, b0, b1);
         const int kt0 = 4 * b0, kt1 = min(KT, 4 * b1);
         for (int kt = kt0; kt < kt1; ++kt, ++it) {
           const int s = static_cast<int>(it % S);
@@ -396,7 +460,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr int kVec = 16 / sizeof(OutT);  // outputs per 16-byte store
       OutT* stg = reinterpret_cast<OutT*>(epi_st + (warp - kWarpEpi0) * kEpiStageBytes);  // [32 tokens][32 rows]
       const bool ld_ok = (p.ld_out % kVec) == 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int r = q * 32 + lane;  // row of the tile (TMEM lane)
+      uint32_t epi_phase = 0, sk_phase = 0;
+      auto epi_sync = [&]() -> bool {
+        mbar_arrive(epi_bar);
+        return mbar_wait_bounded(epi_bar, (epi_phase++) & 1, abort_flag, p.status);
+      };
+      for (int64_t wc = work_first; work_valid(wc); ++local) {
+        int tile, b0, b1;
+        work_get(wc, tile, b0, b1);
+        wc = work_next(wc, b0, b1);
         const uint32_t buf = local % C::kAccBufs;
         const int m0 = (tile % m_tiles) * kBM;
         const int n0 = (tile / m_tiles) * NTILE;
@@ -405,12 +478,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float rs = (row < p.M) ? __half2float(p.rowscale[row]) : 0.f;  // in flight during the wait
         if (!mbar_wait_bounded(&acc_full[buf], (local / C::kAccBufs) & 1, abort_flag, p.status)) break;
         tc_fence_after();
+        const uint32_t acc_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * NTILE;
+        if (SK && b0 > 0) {
+          // stream-K, a later part of a tile: leave the fp32 partial in this
+          // CTA's slot, [column / 4][row] float4, and raise the slot's flag
+          float4* slot = reinterpret_cast<float4*>(p.sk_slots) + static_cast<size_t>(blockIdx.x) * (kSkSlotBytes / 16);
+          for (int col = 0; col < NTILE; col += 32) {
+            if (n0 + col >= p.batch) break;  // warp-uniform
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(acc_addr + static_cast<uint32_t>(col), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              slot[(col / 4 + i) * kBM + r] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                          __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+          if (!epi_sync()) break;  // every epilogue thread's part is stored
+          if (tid == kWarpEpi0 * 32) {
+            __threadfence();
+            st_release_gpu_u32(p.sk_flags + blockIdx.x, 1u);
+          }
+          continue;
+        }
+        // stream-K, the first part of a tile that later CTAs finish
+        // (contributors blockIdx.x+1 .. c_end-1): the MMAs are done, so the B
+        // ring is idle; each contributor's partial is bulk-copied into it and
+        // added into the accumulator in TMEM, in CTA order
+        int c_end = static_cast<int>(blockIdx.x) + 1;
+        bool parts_ok = true;
+        if (SK && b1 < nblk) {
+          const int64_t tile_end = static_cast<int64_t>(tile + 1) * nblk;
+          while (c_end < static_cast<int>(gridDim.x) && sk_lo(c_end) < tile_end) ++c_end;
+          const int ncols = min(NTILE, (p.batch - n0 + 31) / 32 * 32);  // the columns the parts hold
+          const uint32_t bytes = static_cast<uint32_t>(ncols) * kBM * 4;
+          const float4* part = reinterpret_cast<const float4*>(b_st);
+          for (int c = static_cast<int>(blockIdx.x) + 1; c < c_end && parts_ok; ++c) {
+            if (tid == kWarpEpi0 * 32 && flag_wait_bounded(p.sk_flags + c, abort_flag, p.status)) {
+              fence_proxy_async_global();  // the part was written through the generic proxy
+              mbar_arrive_expect_tx(sk_bar, bytes);
+              const char* src = reinterpret_cast<const char*>(p.sk_slots) + static_cast<size_t>(c) * kSkSlotBytes;
+              for (uint32_t off = 0; off < bytes; off += 32768u)
+                bulk_load(b_st + off, src + off, bytes - off < 32768u ? bytes - off : 32768u, sk_bar);
+            }
+            parts_ok = mbar_wait_bounded(sk_bar, (sk_phase++) & 1, abort_flag, p.status);
+            if (!parts_ok) break;
+            for (int col = 0; col < ncols; col += 32) {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(acc_addr + static_cast<uint32_t>(col), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 t = part[(col / 4 + i) * kBM + r];
+                v[4 * i] = __float_as_uint(__uint_as_float(v[4 * i]) + t.x);
+                v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) + t.y);
+                v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) + t.z);
+                v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) + t.w);
+              }
+              tmem_st_32x32b_x32(acc_addr + static_cast<uint32_t>(col), v);
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();  // these reads come before the next copy into the ring
+            parts_ok = epi_sync();
+          }
+        }
         const bool rows_full = row0 + 32 <= p.M;
-        for (int col = 0; col < NTILE; col += 32) {
+        for (int col = 0; col < NTILE && parts_ok; col += 32) {
           if (n0 + col >= p.batch) break;  // warp-uniform
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * NTILE + static_cast<uint32_t>(col),
-                             v);
+          tmem_ld_32x32b_x32(acc_addr + static_cast<uint32_t>(col), v);
           tmem_ld_wait();
           const int tok0 = n0 + col;
           if (rows_full && ld_ok && tok0 + 32 <= p.batch) {
@@ -451,6 +588,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);
+        if (!parts_ok) break;
+        if (SK && c_end > static_cast<int>(blockIdx.x) + 1) {
+          if (!epi_sync()) break;  // every epilogue thread has read the partials
+          if (tid == kWarpEpi0 * 32)
+            for (int c = static_cast<int>(blockIdx.x) + 1; c < c_end; ++c) p.sk_flags[c] = 0u;  // zero for the next launch
+        }
       }
     }
   }
@@ -618,10 +761,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32, bool ATMEM>
+template <int NTILE, bool SPLIT, bool KSCALE, bool OUT_F32, bool ATMEM, bool SK>
 dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, const DeviceInfo& dev,
                         cudaStream_t stream) {
-  auto kernel = dbf_prefill_gemm_kernel<NTILE, SPLIT, KSCALE, OUT_F32, ATMEM>;
+  auto kernel = dbf_prefill_gemm_kernel<NTILE, SPLIT, KSCALE, OUT_F32, ATMEM, SK>;
   constexpr int smem = Cfg<NTILE, SPLIT, ATMEM>::kSmemBytes;
   static std::once_flag once;  // the attribute once per instantiation
   static cudaError_t attr_err = cudaSuccess;
@@ -629,8 +772,11 @@ dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, co
   if (attr_err != cudaSuccess) return DBF_ERR_CUDA;
   const int64_t m_tiles = (a.M + kBM - 1) / kBM;
   const int64_t n_tiles = (a.batch + NTILE - 1) / NTILE;
-  // split K: one (tile, K slice) item per CTA, the ks slices of a tile in one cluster
-  const int64_t grid = SPLIT ? m_tiles * n_tiles * ks : std::min<int64_t>(m_tiles * n_tiles, dev.num_sms);
+  // split K: one (tile, K slice) item per CTA, the ks slices of a tile in one
+  // cluster; stream-K: one range of units per SM (all CTAs resident at once)
+  const int64_t grid = SPLIT ? m_tiles * n_tiles * ks
+                       : SK  ? std::min<int64_t>(dev.num_sms, kSkMaxCtas)
+                             : std::min<int64_t>(m_tiles * n_tiles, dev.num_sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -648,14 +794,14 @@ dbf_status launch_typed(const PrefillArgs& a, const CUtensorMap& map, int ks, co
   return cudaLaunchKernelEx(&cfg, kernel, map, a) == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
-template <int NTILE, bool SPLIT, bool ATMEM>
+template <int NTILE, bool SPLIT, bool ATMEM, bool SK = false>
 dbf_status launch_split(const PrefillArgs& a, const CUtensorMap& map, int ks, bool out_f32, const DeviceInfo& dev,
                         cudaStream_t stream) {
   if (a.kscale != nullptr)
-    return out_f32 ? launch_typed<NTILE, SPLIT, true, true, ATMEM>(a, map, ks, dev, stream)
-                   : launch_typed<NTILE, SPLIT, true, false, ATMEM>(a, map, ks, dev, stream);
-  return out_f32 ? launch_typed<NTILE, SPLIT, false, true, ATMEM>(a, map, ks, dev, stream)
-                 : launch_typed<NTILE, SPLIT, false, false, ATMEM>(a, map, ks, dev, stream);
+    return out_f32 ? launch_typed<NTILE, SPLIT, true, true, ATMEM, SK>(a, map, ks, dev, stream)
+                   : launch_typed<NTILE, SPLIT, true, false, ATMEM, SK>(a, map, ks, dev, stream);
+  return out_f32 ? launch_typed<NTILE, SPLIT, false, true, ATMEM, SK>(a, map, ks, dev, stream)
+                 : launch_typed<NTILE, SPLIT, false, false, ATMEM, SK>(a, map, ks, dev, stream);
 }
 
 }  // namespace
@@ -724,7 +870,7 @@ static int max_resident_clusters(int device, int ks, int num_sms) {
   const auto key = std::make_pair(device, ks);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  auto kernel = dbf_prefill_gemm_kernel<128, true, false, false, true>;
+  auto kernel = dbf_prefill_gemm_kernel<128, true, false, false, true, false>;
   constexpr int smem = Cfg<128, true, true>::kSmemBytes;
   int n = 0;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
@@ -752,6 +898,7 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
                                const DeviceInfo& dev, cudaStream_t stream) {
   auto encode = encode_fn();
   if (!encode) return DBF_ERR_CUDA;
+
   int ks = prefill_k_split(a.M, a.K, a.batch, dev.num_sms);
   const int64_t tiles128 = static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + 127) / 128);
   while (ks > 1 && tiles128 > max_resident_clusters(dev.device, ks, dev.num_sms)) ks /= 2;
@@ -765,6 +912,32 @@ dbf_status launch_prefill_gemm(const PrefillArgs& a, const __half* act, int64_t 
   }
   if (static_cast<int64_t>(a.M + kBM - 1) / kBM * ((a.batch + ntile - 1) / ntile) * ks > 0x7fffffffLL)
     return DBF_ERR_UNSUPPORTED_SHAPE;
+
+  // Stream-K past 128 tokens (when the workspace holds its partial-tile slots):
+  // the 256-token tiles' (tile, 256-column block) units cut evenly over the
+  // SMs.  Chosen where its estimated time beats the plan above, counted in
+  // 256 x 256-column block times: stream-K takes units / SMs plus about 5 for
+  // its partial tiles (measured: one partial write, one bulk-copied add and
+  // the extra epilogue drains per CTA); the plan above takes its rounds of
+  // tiles times the blocks per tile, a 128-token tile about 0.77 of a
+  // 256-token one (half the work at a lower tensor-pipe rate), a K slice of
+  // a cluster split 1/ks of a tile.
+  if (a.batch > 128 && a.sk_slots != nullptr && a.sk_flags != nullptr) {
+    const int64_t grid = std::min(dev.num_sms, kSkMaxCtas);
+    const int64_t m_tiles = (a.M + kBM - 1) / kBM;
+    const int64_t nblk = (a.K / kBK + 3) / 4;
+    const int64_t units = m_tiles * ((a.batch + 255) / 256) * nblk;
+    const int64_t plan_items = m_tiles * ((a.batch + ntile - 1) / ntile) * ks;
+    const int64_t plan_rounds = (plan_items + dev.num_sms - 1) / dev.num_sms;
+    const double plan_t = static_cast<double>(plan_rounds) * static_cast<double>(nblk) / ks * (ntile == 128 ? 0.77 : 1.0);
+    const double sk_t = static_cast<double>(units) / static_cast<double>(grid) + 5.0;
+    if (units >= grid && sk_t < 0.95 * plan_t) {
+      CUtensorMap map;
+      if (!activation_map(act, a.K, act_rows, 256, encode, &map)) return DBF_ERR_CUDA;
+      return out_f32 ? launch_split<256, false, false, true>(a, map, 1, true, dev, stream)
+                     : launch_split<256, false, true, true>(a, map, 1, false, dev, stream);
+    }
+  }
 
   // Wave tail.  Without a split the persistent CTAs walk the tiles in waves of
   // one tile per SM, and a last, nearly empty wave costs a whole tile time (896

@@ -136,12 +136,23 @@ DBF_API dbf_status dbf_pack_signs(const void* src, dbf_dtype src_t, int64_t rows
                           uint32_t* packed, struct CUstream_st* stream);
 
 /*
- * Workspace bytes dbf_forward needs for these sizes (0 if a size is < 1).
- * Layout: a 256-byte status block (an int32 status word at offset 0), then
- * the middle activations V = fp16(mid (.) (B (x (.) b))) as batch x k fp16.
- * The workspace must be zero-filled before its first use; the library leaves
- * the status word untouched unless a device-side wait gives up.  Calls that
- * may run concurrently need distinct workspaces.
+ * Workspace bytes that let dbf_forward run every schedule for these sizes
+ * (0 if a size is < 1).  Layout: a 256-byte status block (an int32 status
+ * word at offset 0); the middle activations V = fp16(mid (.) (B (x (.) b))) as
+ * batch x k fp16, padded to 256 bytes; then an optional area:
+ *   batch <= 16: the single-launch decode's tagged partials, 8 x batch x n
+ *                64-bit words (used with DBF_FWD_DECODE_SINGLE);
+ *   batch > 128: the tensor-core path's stream-K area, 1 KiB of flags and 160
+ *                partial tiles of 128 x 256 fp32 (20,972,544 bytes), used for
+ *                the GEMMs whose tiles would leave a partial last wave.
+ * dbf_forward accepts any workspace of at least 256 + round_up(batch*k*2, 256)
+ * bytes and runs a schedule that needs no optional area when it is smaller
+ * than this size.
+ * The workspace must be zero-filled before its first use.  After a call that
+ * leaves the status word at 0 it can be reused as it is (the library returns
+ * every flag it raises to zero; the status word changes only when a
+ * device-side wait gives up, after which the workspace must be zero-filled
+ * again).  Calls that may run concurrently need distinct workspaces.
  */
 DBF_API size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, int64_t batch);
 
@@ -156,8 +167,9 @@ DBF_API size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, i
  *              vector, "mid" above).
  *   y          batch x n, row-major, y_t = DBF_F16 (round to nearest even,
  *              overflow to +-inf) or DBF_F32.
- *   workspace  ws_bytes >= dbf_forward_workspace_bytes(n, k, m_in, batch),
- *              zero-filled before its first use (see above).
+ *   workspace  ws_bytes >= 256 + round_up(batch*k*2, 256); the size
+ *              dbf_forward_workspace_bytes(n, k, m_in, batch) enables every
+ *              schedule.  Zero-filled before its first use (see above).
  *   flags      DBF_FWD_* bits.
  * Arithmetic: both sign products accumulate in fp32.  The middle vector V is
  * rounded to fp16 once (V = fp16(mid (.) t)); the decode path also rounds
@@ -167,7 +179,16 @@ DBF_API size_t dbf_forward_workspace_bytes(int64_t n, int64_t k, int64_t m_in, i
  * Paths: batch <= 16 runs two PDL-chained sign-GEMV kernels (mma.sync);
  * larger batches run the two products as tcgen05 tensor-core GEMMs, one
  * launch each, or two when a GEMM's last wave of tiles would leave most SMs
- * idle (its last rows then run as a split-K launch of their own).
+ * idle (its last rows then run as a split-K launch of their own).  Past 128
+ * tokens a GEMM whose tiles do not fill whole waves may instead run stream-K
+ * (one contiguous range of (tile, K block) units per SM; a tile split between
+ * CTAs is completed by the CTA holding its first K blocks, which adds the
+ * others' fp32 partial tiles in a fixed order): results then differ from the
+ * one-launch schedule only in the grouping of fp32 additions, and are
+ * identical in integer mode.  Stream-K waits on other CTAs of its own grid
+ * (bounded, DBF_ERR_TIMEOUT): its CTAs, one per SM, must all become resident
+ * within the wait budget, so it should not share the GPU with kernels that
+ * hold SMs for longer.
  * Shape contract: n >= 1, batch >= 1, k and m_in multiples of 64 in
  * [64, 1 << 20], n and batch <= 1 << 24.  All pointers 16-byte aligned;
  * outputs must not overlap inputs.
@@ -207,10 +228,11 @@ DBF_API dbf_status dbf_workspace_status(const void* workspace, struct CUstream_s
  * dbf_forward minus the workspace and uses instead a 2 MiB buffer that lives
  * in the library (a static __device__ array, held by every GPU that loads the
  * library until the process exits).  It allocates and frees nothing.
- *   Limit: dbf_forward_workspace_bytes(n, k, m_in, batch) <= 2 MiB, i.e.
- *   256 + batch*k*2 bytes (e.g. batch 16 with k up to 65472, or batch 256 with
- *   k up to 4032, k being a multiple of 64); larger sizes return
- *   DBF_ERR_WORKSPACE.
+ *   Limit: the smallest workspace dbf_forward accepts, 256 + batch*k*2 bytes
+ *   (rounded up to 256), must fit in 2 MiB (e.g. batch 16 with k up to 65472,
+ *   or batch 256 with k up to 4032, k being a multiple of 64); larger sizes
+ *   return DBF_ERR_WORKSPACE.  The optional areas do not fit, so this call
+ *   runs the schedules that need none (no single-launch decode, no stream-K).
  *   The first call on each device looks up the buffer's device address with
  *   that device current; make that first call before any stream capture.  A
  *   failed lookup (DBF_ERR_CUDA) is not remembered: the next call retries.
@@ -253,8 +275,9 @@ DBF_API dbf_status dbf_noalloc_status(struct CUstream_st* stream, int32_t* devic
  *              over the shared m_in; y: batch x n output of layer g
  *              (row-major, y_t).  The array is read during the call only.
  *   num_layers 1 .. DBF_MAX_GROUP.
- *   workspace  ws_bytes >= dbf_forward_grouped_workspace_bytes(...) for the
- *              same layers, zero-filled before its first use.
+ *   workspace  ws_bytes >= 256 + sum over layers of round_up(batch * k_g * 2,
+ *              256); dbf_forward_grouped_workspace_bytes(...) adds the
+ *              stream-K area past 128 tokens.  Zero-filled before its first use.
  * Per-layer results equal dbf_forward's up to the order of fp32 additions
  * (the K split can differ); in integer mode they are identical.
  * Shape contract per layer as dbf_forward; flags as dbf_forward.
@@ -272,7 +295,9 @@ typedef struct dbf_layer_desc {
 } dbf_layer_desc;
 
 /* Workspace bytes for dbf_forward_grouped (0 if an argument is out of range):
- * 256 + sum over layers of round_up(batch * k_g * 2, 256). */
+ * 256 + sum over layers of round_up(batch * k_g * 2, 256), plus past 128
+ * tokens the stream-K area of dbf_forward_workspace_bytes (shared by the
+ * layers, which run one after another). */
 DBF_API size_t dbf_forward_grouped_workspace_bytes(const dbf_layer_desc* layers, int num_layers, int64_t m_in,
                                                    int64_t batch);
 

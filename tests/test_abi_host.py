@@ -62,6 +62,9 @@ def test_workspace_bytes(lib):
     assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 4) == 256 + 1024 + 8 * 4 * 256 * 8
     assert dbf.dbf_forward_workspace_bytes(256, 64, 256, 1) == 256 + 256 + 8 * 256 * 8
     assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 17) == 256 + 17 * 256  # no partials past 16 tokens
+    assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 128) == 256 + 128 * 256
+    # past 128 tokens: the stream-K area (1 KiB of flags, 160 partial tiles of 128 x 256 fp32) after V
+    assert dbf.dbf_forward_workspace_bytes(256, 128, 256, 129) == 256 + 129 * 256 + 1024 + 160 * 128 * 256 * 4
     assert dbf.dbf_forward_workspace_bytes(0, 128, 256, 4) == 0
 
 
@@ -160,6 +163,9 @@ def test_grouped_workspace_bytes(lib):
     assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=256, k=128), dict(n=64, k=64)], 256, 4) == \
         256 + 1024 + 512
     assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=8, k=832)], 4096, 3) == 256 + 5120
+    # past 128 tokens the stream-K area follows the V blocks
+    assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=8, k=64)], 64, 200) == \
+        256 + 200 * 128 + 1024 + 160 * 128 * 256 * 4
     assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=0, k=64)], 64, 1) == 0
     assert dbf.dbf_forward_grouped_workspace_bytes([dict(n=1, k=64)] * 9, 64, 1) == 0
 
