@@ -25,7 +25,7 @@ __all__ = [
     "DBFError",
     "DBF_I8", "DBF_F16", "DBF_F32",
     "DBF_FWD_WEIGHTS_STATIC", "DBF_FWD_FORCE_DECODE", "DBF_FWD_FORCE_PREFILL", "DBF_FWD_DECODE_SHIFT_EXPAND",
-    "DBF_FWD_DECODE_TWO_STAGE", "DBF_FWD_DECODE_SINGLE", "DBF_FWD_TEST_LOSE_ARRIVAL",
+    "DBF_FWD_DECODE_TWO_STAGE", "DBF_FWD_DECODE_SINGLE", "DBF_FWD_DECODE_TABLE", "DBF_FWD_TEST_LOSE_ARRIVAL",
     "EXPORTED_SYMBOLS",
     "library_path", "load_library",
     "dbf_packed_words_per_row", "dbf_packed_words", "dbf_pack_signs",
@@ -46,6 +46,7 @@ DBF_FWD_FORCE_PREFILL = 1 << 2
 DBF_FWD_DECODE_SHIFT_EXPAND = 1 << 3
 DBF_FWD_DECODE_TWO_STAGE = 1 << 4
 DBF_FWD_DECODE_SINGLE = 1 << 5
+DBF_FWD_DECODE_TABLE = 1 << 6
 DBF_FWD_TEST_LOSE_ARRIVAL = 1 << 30  # test only: makes a bounded device wait run out
 
 STATUS_NAMES = {

@@ -140,10 +140,13 @@ dbf_status validate_forward_args(const uint16_t* x, const uint32_t* packedA, con
   if (y_t != DBF_F16 && y_t != DBF_F32) return DBF_ERR_INVALID_ARG;
   const uint32_t known = DBF_FWD_WEIGHTS_STATIC | DBF_FWD_FORCE_DECODE | DBF_FWD_FORCE_PREFILL |
                          DBF_FWD_DECODE_SHIFT_EXPAND | DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SINGLE |
+                         DBF_FWD_DECODE_TABLE |
                          DBF_FWD_TEST_LOSE_ARRIVAL;
   if ((flags & ~known) != 0) return DBF_ERR_INVALID_ARG;
-  if ((flags & DBF_FWD_DECODE_SINGLE) && (flags & (DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SHIFT_EXPAND)))
+  if ((flags & DBF_FWD_DECODE_SINGLE) &&
+      (flags & (DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SHIFT_EXPAND | DBF_FWD_DECODE_TABLE)))
     return DBF_ERR_INVALID_ARG;
+  if ((flags & DBF_FWD_DECODE_TABLE) && (flags & DBF_FWD_DECODE_SHIFT_EXPAND)) return DBF_ERR_INVALID_ARG;
   if ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)) return DBF_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return DBF_ERR_MISALIGNED;
   return DBF_OK;
@@ -177,6 +180,8 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
   const bool decode = (flags & DBF_FWD_FORCE_DECODE) || (!(flags & DBF_FWD_FORCE_PREFILL) && batch <= 16);
   if (decode) {
     const bool class_expand = (flags & DBF_FWD_DECODE_SHIFT_EXPAND) == 0;
+    // one token: the lookup-table kernel when asked for
+    const bool lut = (flags & DBF_FWD_DECODE_TABLE) != 0;
     // the single-launch kernel when asked for (its measured per-layer time
     // does not yet beat the two launches on any layer shape of the workloads)
     const bool two_stage = (flags & DBF_FWD_DECODE_SINGLE) == 0;
@@ -222,7 +227,7 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
       sb.weights_early = early ? 1 : 0;
       sb.peer_rows = static_cast<int>(n);
       sb.status = status;
-      st = launch_decode_stage(sb, class_expand, /*out_f32=*/false, dev, stream);
+      st = launch_decode_stage(sb, class_expand, lut, /*out_f32=*/false, dev, stream);
       if (st != DBF_OK) return st;
       DecodeArgs sa{};
       sa.packed = packedA;
@@ -239,7 +244,7 @@ dbf_status dbf_forward(const uint16_t* x, const uint32_t* packedA, const uint32_
       sa.weights_early = 1;  // stage B releases stage A only after its own wait
       sa.peer_rows = static_cast<int>(k);
       sa.status = status;
-      st = launch_decode_stage(sa, class_expand, out_f32, dev, stream);
+      st = launch_decode_stage(sa, class_expand, lut, out_f32, dev, stream);
       if (st != DBF_OK) return st;
     }
     return DBF_OK;
@@ -312,8 +317,10 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
   if (y_t != DBF_F16 && y_t != DBF_F32) return DBF_ERR_INVALID_ARG;
   // (the grouped decode always runs the two-launch kernels: DBF_FWD_DECODE_TWO_STAGE changes nothing here)
   const uint32_t known = DBF_FWD_WEIGHTS_STATIC | DBF_FWD_FORCE_DECODE | DBF_FWD_FORCE_PREFILL |
-                         DBF_FWD_DECODE_SHIFT_EXPAND | DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SINGLE;
+                         DBF_FWD_DECODE_SHIFT_EXPAND | DBF_FWD_DECODE_TWO_STAGE | DBF_FWD_DECODE_SINGLE |
+                         DBF_FWD_DECODE_TABLE;
   if ((flags & ~known) != 0) return DBF_ERR_INVALID_ARG;
+  if ((flags & DBF_FWD_DECODE_TABLE) && (flags & DBF_FWD_DECODE_SHIFT_EXPAND)) return DBF_ERR_INVALID_ARG;
   if ((flags & DBF_FWD_FORCE_DECODE) && (flags & DBF_FWD_FORCE_PREFILL)) return DBF_ERR_INVALID_ARG;
   if (!aligned16(x)) return DBF_ERR_MISALIGNED;
   if (!workspace || !aligned16(workspace) || ws_bytes < grouped_v_offset(layers, num_layers, batch))
@@ -339,6 +346,7 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
   const bool decode = (flags & DBF_FWD_FORCE_DECODE) || (!(flags & DBF_FWD_FORCE_PREFILL) && batch <= 16);
   if (decode) {
     const bool class_expand = (flags & DBF_FWD_DECODE_SHIFT_EXPAND) == 0;
+    const bool lut = (flags & DBF_FWD_DECODE_TABLE) != 0;
     for (int64_t t0 = 0; t0 < batch; t0 += 16) {
       const int nb = static_cast<int>(batch - t0 < 16 ? batch - t0 : 16);
       DecodeGroup gb{};
@@ -375,9 +383,9 @@ dbf_status dbf_forward_grouped(const uint16_t* x, int64_t m_in, int64_t batch, c
         sa.weights_early = 1;  // the stage-B launch releases this one only after its own wait
         sa.status = status;
       }
-      st = launch_decode_group(gb, rows_a, class_expand, /*out_f32=*/false, dev, stream);
+      st = launch_decode_group(gb, rows_a, class_expand, lut, /*out_f32=*/false, dev, stream);
       if (st != DBF_OK) return st;
-      st = launch_decode_group(ga, rows_b, class_expand, out_f32, dev, stream);
+      st = launch_decode_group(ga, rows_b, class_expand, lut, out_f32, dev, stream);
       if (st != DBF_OK) return st;
     }
     return DBF_OK;

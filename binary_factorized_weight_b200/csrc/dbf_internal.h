@@ -73,7 +73,7 @@ dbf_status validate_forward_args(const uint16_t* x, const uint32_t* packedA, con
                                  const uint16_t* a, const uint16_t* m, const uint16_t* b, int64_t n, int64_t k,
                                  int64_t m_in, int64_t batch, const void* y, dbf_dtype y_t, uint32_t flags);
 
-dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
+dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool lut, bool out_f32, const DeviceInfo& dev,
                                cudaStream_t stream);
 
 // Several decode stages in one launch (layers that share their input: the
@@ -90,7 +90,7 @@ struct DecodeGroup {
 
 // Fills tile_start and each layer's kchunk, then launches.  peer_rows: rows of
 // the forward's other stage (all layers).
-dbf_status launch_decode_group(DecodeGroup& group, int64_t peer_rows, bool class_expand, bool out_f32,
+dbf_status launch_decode_group(DecodeGroup& group, int64_t peer_rows, bool class_expand, bool lut, bool out_f32,
                                const DeviceInfo& dev, cudaStream_t stream);
 
 // The single-launch decode forward (fused.cu): grid (R, J), clusters of R

@@ -486,6 +486,261 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- one token: table lookup
+//
+// With a single token an MMA carries one useful column of eight, so the sums
+// are formed by table lookup instead: for each nibble of a packed word (four
+// sign bits) the CTA builds, once per piece of K, a table of the 16 signed
+// sums of the four activations those bits select, and a row's product is the
+// sum of one table entry per nibble of its words.  In the packed layout bit i
+// of nibble j of word p of a 256-column block is the column
+//   16 (4 (j mod 4) + i) + 2p + (j div 4),
+// so table (block, p, j) holds T[v] = sum_i (bit i of v ? -u : u)[column_i].
+// Tables are fp32 built from u = x (.) b in fp32 (exact for fp16 x and b), so
+// this path does not round u to fp16.  Lane = weight row: all 32 lanes of a
+// warp read the same 16-entry table at a time (conflict-free).  A CTA has 64
+// rows: warp w takes rows 32 (w / 2) .. + 31 and half (w mod 2) of the blocks
+// of each piece; K is split over a cluster as in the MMA kernel and the
+// partials meet in rank 0 (rank-major, half minor: a fixed order).
+constexpr int kLutD = 4;  // blocks of weights per register group
+
+struct LutSmem {
+  int act_off, b_off, tab_off, rs_off, red_off, total;
+};
+
+__host__ __device__ inline LutSmem lut_smem_layout(int piece, int ks) {
+  LutSmem l;
+  l.act_off = kHeadBytes;
+  l.b_off = l.act_off + piece * 2;
+  l.tab_off = (l.b_off + piece * 2 + 15) / 16 * 16;
+  l.rs_off = l.tab_off + piece * 16;  // piece / 4 tables of 16 fp32
+  l.red_off = l.rs_off + 64 * 4;
+  l.total = l.red_off + ks * 2 * 64 * 4;
+  return l;
+}
+
+template <bool KSCALE, bool OUT_F32>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    dbf_decode_lut_kernel(const __grid_constant__ DecodeGroup grp, const int piece) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  int li = 0;
+  while (li + 1 < grp.n && static_cast<int>(blockIdx.x) >= grp.tile_start[li + 1]) ++li;
+  const DecodeArgs& p = grp.layer[li];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int ks = static_cast<int>(cluster.num_blocks());
+  const LutSmem L = lut_smem_layout(piece, ks);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + 16);
+  uint64_t* bar_red = reinterpret_cast<uint64_t*>(smem + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 8);
+  __half* act_s = reinterpret_cast<__half*>(smem + L.act_off);
+  __half* b_s = reinterpret_cast<__half*>(smem + L.b_off);
+  float* tab_s = reinterpret_cast<float*>(smem + L.tab_off);
+  float* rs_s = reinterpret_cast<float*>(smem + L.rs_off);
+  float* red_s = reinterpret_cast<float*>(smem + L.red_off);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int rg = warp >> 1, half = warp & 1;
+  const int m0 = (static_cast<int>(blockIdx.x) - grp.tile_start[li]) * 64;
+  const int row = m0 + 32 * rg + lane;
+  const bool rok = row < p.M;
+  const int k_lo = rank * p.kchunk;
+  const int k_hi = min(p.K, k_lo + p.kchunk);
+  const uint4* wrow = reinterpret_cast<const uint4*>(p.packed + static_cast<int64_t>(rok ? row : 0) * p.wpr);
+
+  // this warp's blocks of a piece [pk, pe): its half of the piece's blocks
+  auto slice = [&](int pk, int pe, int& b0, int& b1) {
+    const int pb0 = pk >> 8, pb1 = (pe + 255) >> 8;
+    const int per = (pb1 - pb0 + 1) / 2;
+    b0 = min(pb1, pb0 + half * per);
+    b1 = min(pb1, b0 + per);
+  };
+  uint4 wa[kLutD][2], wb[kLutD][2];
+  auto load_group = [&](uint4 (&wr)[kLutD][2], int blk0, int blk_end) {
+#pragma unroll
+    for (int d = 0; d < kLutD; ++d) {
+      const bool in = rok && blk0 + d < blk_end;
+      wr[d][0] = in ? __ldg(wrow + 2 * (blk0 + d)) : make_uint4(0u, 0u, 0u, 0u);
+      wr[d][1] = in ? __ldg(wrow + 2 * (blk0 + d) + 1) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  auto load_static = [&](int pk, int pe) {
+    if (tid < 64) rs_s[tid] = (m0 + tid < p.M) ? __half2float(p.rowscale[m0 + tid]) : 0.f;
+    if constexpr (KSCALE) {
+      if (tid == 0 && pe > pk) {
+        const uint32_t bytes = static_cast<uint32_t>(pe - pk) * 2;
+        mbar_arrive_expect_tx(bar_b, bytes);
+        bulk_load(b_s, p.kscale + pk, bytes, bar_b);
+      }
+    }
+  };
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar_b, 1);
+    mbar_init(bar_red, ks > 1 ? (ks - 1) * kDecThreads : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (ks > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+
+  int pk = k_lo;
+  int pe = min(k_hi, pk + piece);
+  int sb0, sb1;
+  slice(pk, pe, sb0, sb1);
+  if (p.weights_early) {
+    load_group(wa, sb0, sb1);
+    load_static(pk, pe);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!p.weights_early) {
+    load_group(wa, sb0, sb1);
+    load_static(pk, pe);
+  }
+
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  bool ok = true;
+  uint32_t phase = 0;
+  const bool has_k = k_lo < k_hi;
+  while (has_k) {
+    const int plen = pe - pk;  // multiple of 64
+    if (tid == 0) {
+      const uint32_t bytes = static_cast<uint32_t>(plen) * 2;
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_load(act_s, p.act + pk, bytes, bar);
+    }
+    ok = mbar_wait_bounded(bar, phase, abort_flag, p.status);
+    if constexpr (KSCALE) ok = ok && mbar_wait_bounded(bar_b, phase, abort_flag, p.status);
+    phase ^= 1u;
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+
+    // ---- the tables of this piece: table tb = (block, word p, nibble j)
+    const int ntab = ((plen + 255) >> 8) * 64;
+    for (int tb = tid; tb < ntab; tb += kDecThreads) {
+      const int pw = (tb >> 3) & 7, j = tb & 7;
+      const int base = (tb >> 6) * 256 + 2 * pw + (j >> 2) + 64 * (j & 3);
+      float u[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = base + 16 * i;
+        float v = 0.f;
+        if (col < plen) {
+          v = __half2float(act_s[col]);
+          if constexpr (KSCALE) v *= __half2float(b_s[col]);
+        }
+        u[i] = v;
+      }
+      // v = bits (b0 b1 b2 b3): e[v & 3] + f[v >> 2], a set bit negating its term
+      const float e0 = u[0] + u[1], e1 = u[1] - u[0], e2 = u[0] - u[1], e3 = -(u[0] + u[1]);
+      const float f0 = u[2] + u[3], f1 = u[3] - u[2], f2 = u[2] - u[3], f3 = -(u[2] + u[3]);
+      float4* t4 = reinterpret_cast<float4*>(tab_s + tb * 16);
+      t4[0] = make_float4(e0 + f0, e1 + f0, e2 + f0, e3 + f0);
+      t4[1] = make_float4(e0 + f1, e1 + f1, e2 + f1, e3 + f1);
+      t4[2] = make_float4(e0 + f2, e1 + f2, e2 + f2, e3 + f2);
+      t4[3] = make_float4(e0 + f3, e1 + f3, e2 + f3, e3 + f3);
+    }
+    __syncthreads();
+
+    // ---- one lookup per nibble of this lane's words
+    const int pb0 = pk >> 8;
+    for (int gb = sb0; gb < sb1; gb += kLutD) {
+      if (gb + kLutD < sb1) load_group(wb, gb + kLutD, sb1);
+#pragma unroll
+      for (int d = 0; d < kLutD; ++d) {
+        if (gb + d < sb1) {
+          const float* tblk = tab_s + (gb + d - pb0) * 64 * 16;
+          const uint32_t wd[8] = {wa[d][0].x, wa[d][0].y, wa[d][0].z, wa[d][0].w,
+                                  wa[d][1].x, wa[d][1].y, wa[d][1].z, wa[d][1].w};
+#pragma unroll
+          for (int pw = 0; pw < 8; ++pw) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j & 3] += tblk[(pw * 8 + j) * 16 + ((wd[pw] >> (4 * j)) & 15u)];
+          }
+        }
+      }
+#pragma unroll
+      for (int d = 0; d < kLutD; ++d) {
+        wa[d][0] = wb[d][0];
+        wa[d][1] = wb[d][1];
+      }
+    }
+
+    pk = pe;
+    if (pk >= k_hi) break;
+    pe = min(k_hi, pk + piece);
+    fence_proxy_async_smem();  // this piece's shared reads before the next bulk copies overwrite it
+    __syncthreads();
+    slice(pk, pe, sb0, sb1);
+    load_group(wa, sb0, sb1);
+    load_static(pk, pe);
+  }
+
+  // ---- this warp's partial of its 32 rows, to rank 0
+  const int slot = rank * 2 + half;
+  if (ks > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  {
+    const float t = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    float* dst = &red_s[slot * 64 + 32 * rg + lane];
+    if (rank == 0) {
+      *dst = t;
+    } else {
+      st_cluster_f32(map_to_rank(dst, 0), t);
+    }
+  }
+  if (ks > 1 && rank != 0) {
+    mbar_arrive_remote_release(map_to_rank(bar_red, 0));
+    return;
+  }
+  __syncthreads();
+  if (ks > 1) ok = mbar_wait_cluster_bounded(bar_red, 0, p.status) && ok;
+  if (rank == 0 && ok && tid < 64) {
+    const int r = m0 + tid;
+    if (r < p.M) {
+      float t = 0.f;
+      for (int q = 0; q < 2 * ks; ++q) t += red_s[q * 64 + tid];
+      const float v = t * rs_s[tid];
+      if constexpr (OUT_F32) {
+        static_cast<float*>(p.out)[r] = v;
+      } else {
+        static_cast<__half*>(p.out)[r] = __float2half_rn(v);
+      }
+    }
+  }
+}
+
+template <bool KSCALE, bool OUT_F32>
+dbf_status launch_lut(const DecodeGroup& grp, int ks, int piece, cudaStream_t stream) {
+  auto kernel = dbf_decode_lut_kernel<KSCALE, OUT_F32>;
+  const size_t smem = static_cast<size_t>(lut_smem_layout(piece, ks).total);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  });
+  if (attr_err != cudaSuccess || smem > static_cast<size_t>(kMaxDynSmem)) return DBF_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grp.tile_start[grp.n]), static_cast<unsigned>(ks), 1);
+  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = 1;
+  attrs[0].val.clusterDim.y = static_cast<unsigned>(ks);
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, grp, piece) == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
+}
+
 template <int NT, int RT, int D, bool TOKPAR, bool CLASS, bool KSCALE, bool OUT_F32>
 dbf_status launch_typed(const DecodeGroup& grp, int batch, int ks, int piece, cudaStream_t stream) {
   auto kernel = dbf_decode_stage_kernel<NT, RT, D, TOKPAR, CLASS, KSCALE, OUT_F32>;
@@ -577,7 +832,7 @@ static DecodePlan plan_decode(int64_t M, int64_t K, int batch, int num_sms, int6
   return DecodePlan{4, ks_eff, piece, kchunk};
 }
 
-dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_expand, bool out_f32,
+dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_expand, bool lut, bool out_f32,
                                const DeviceInfo& dev, cudaStream_t stream) {
   if (grp.n < 1 || grp.n > kMaxGroup) return DBF_ERR_INVALID_ARG;
   const int batch = grp.layer[0].batch;
@@ -599,6 +854,18 @@ dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_e
     int64_t kc = (grp.layer[g].K + plan.ks - 1) / plan.ks;
     grp.layer[g].kchunk = static_cast<int>((kc + 255) / 256 * 256);
   }
+  if (lut && batch == 1) {
+    // one token: the lookup-table kernel (64-row CTAs, the same K split); a
+    // piece is the whole K chunk unless the tables would not fit
+    int kmax_chunk = 0;
+    for (int g = 0; g < grp.n; ++g) kmax_chunk = std::max(kmax_chunk, grp.layer[g].kchunk);
+    int piece = kmax_chunk;
+    while (piece > 256 && lut_smem_layout(piece, plan.ks).total > kSmemBudget) piece -= 256;
+    if (kscale) return out_f32 ? launch_lut<true, true>(grp, plan.ks, piece, stream)
+                               : launch_lut<true, false>(grp, plan.ks, piece, stream);
+    return out_f32 ? launch_lut<false, true>(grp, plan.ks, piece, stream)
+                   : launch_lut<false, false>(grp, plan.ks, piece, stream);
+  }
   int64_t max_blocks = 0;
   for (int g = 0; g < grp.n; ++g) max_blocks = std::max<int64_t>(max_blocks, grp.layer[g].kchunk / 256);
   // 8-block groups cost registers: keep them to launches of at most 1.75 CTAs
@@ -617,12 +884,12 @@ dbf_status launch_decode_group(DecodeGroup& grp, int64_t peer_rows, bool class_e
                    : launch_rt<1, 4, 4, false>(grp, batch, kscale, class_expand, out_f32, plan.ks, plan.piece, stream);
 }
 
-dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool out_f32, const DeviceInfo& dev,
+dbf_status launch_decode_stage(const DecodeArgs& args, bool class_expand, bool lut, bool out_f32, const DeviceInfo& dev,
                                cudaStream_t stream) {
   DecodeGroup grp{};
   grp.n = 1;
   grp.layer[0] = args;
-  return launch_decode_group(grp, args.peer_rows, class_expand, out_f32, dev, stream);
+  return launch_decode_group(grp, args.peer_rows, class_expand, lut, out_f32, dev, stream);
 }
 
 }  // namespace dbf

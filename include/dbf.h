@@ -104,6 +104,14 @@ enum {
    * thread-block clusters) wherever the shape fits it, instead of the
    * library's choice between the two decode kernels. */
   DBF_FWD_DECODE_SINGLE = 1u << 5,
+  /* Decode path, one token: form the products by table lookup instead of the
+   * fp16 warp-MMA sign-GEMV: per nibble of packed signs a table of the 16
+   * signed sums of the four activations it selects, built in fp32 from
+   * u = x (.) b (so u is not rounded to fp16; V still is).  Slower than the
+   * default on most layer shapes, faster on layers of about 1000 rows; no
+   * effect above one token.  Not with DBF_FWD_DECODE_SHIFT_EXPAND or
+   * DBF_FWD_DECODE_SINGLE. */
+  DBF_FWD_DECODE_TABLE = 1u << 6,
   /* TEST ONLY.  Makes one bounded wait of the single-launch decode kernel run
    * out (rank 0 of each cluster waits for 16 bytes that are never sent), so
    * that failure reporting can be tested without a fault: the call still

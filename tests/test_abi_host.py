@@ -94,7 +94,8 @@ def fwd(lib, x=P, A=P, B=P, a=P, m=P, b=P, n=256, k=128, m_in=256, batch=4, y=P,
         (dict(batch=(1 << 24) + 1), SHAPE),
         (dict(y_t=0), INVALID), (dict(y_t=7), INVALID),
         (dict(flags=1 << 9), INVALID), (dict(flags=2 | 4), INVALID), (dict(flags=32 | 16), INVALID),
-        (dict(flags=32 | 8), INVALID),
+        (dict(flags=32 | 8), INVALID), (dict(flags=32 | 64), INVALID), (dict(flags=64 | 8), INVALID),
+        (dict(flags=1 << 7), INVALID),
         (dict(x=MIS), MISALIGNED), (dict(A=MIS), MISALIGNED), (dict(B=MIS), MISALIGNED),
         (dict(a=MIS), MISALIGNED), (dict(y=MIS), MISALIGNED),
         (dict(ws=None), WORKSPACE), (dict(ws=MIS), WORKSPACE), (dict(ws_bytes=256 + 1023), WORKSPACE),

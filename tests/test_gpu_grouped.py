@@ -53,7 +53,7 @@ def make_group(dbf, shapes, m_in, batch, seed, integer=False):
 SMALL = [(256, 128), (64, 64), (128, 192)]
 
 
-@pytest.mark.parametrize("path", ["default", "decode_class", "decode_shift", "prefill"])
+@pytest.mark.parametrize("path", ["default", "decode_class", "decode_shift", "decode_table", "prefill"])
 @pytest.mark.parametrize("batch", [1, 5, 16, 20, 200])
 def test_grouped_integer_bit_exact(dbf, path, batch):
     x, layers, facts = make_group(dbf, SMALL, 256, batch, seed=7, integer=True)
@@ -65,7 +65,7 @@ def test_grouped_integer_bit_exact(dbf, path, batch):
         assert np.array_equal(ys[g].cpu().numpy().astype(np.float64), ref), f"layer {g}"
 
 
-@pytest.mark.parametrize("path", ["default", "decode_class", "prefill"])
+@pytest.mark.parametrize("path", ["default", "decode_class", "decode_table", "prefill"])
 @pytest.mark.parametrize("batch", [1, 9, 16, 130])
 def test_grouped_fp16(dbf, path, batch):
     x, layers, facts = make_group(dbf, SMALL, 256, batch, seed=11)

@@ -94,6 +94,7 @@ def random_layer(dbf, n, k, m_in, batch, seed, scales="absnormal", x_kind="norma
 PATHS = {
     "decode_fused": 2 | 32,  # + DBF_FWD_DECODE_SINGLE: the single-launch int8 kernel where the shape fits
     "decode_class": 2 | 16,  # + DBF_FWD_DECODE_TWO_STAGE: two launches, fp16 class form
+    "decode_table": 2 | 16 | 64,  # + DBF_FWD_DECODE_TABLE: two launches, one token by table lookup (class form above)
     "decode_shift": 2 | 8,  # + DBF_FWD_DECODE_SHIFT_EXPAND (two launches, shift form)
     "prefill": 4,  # DBF_FWD_FORCE_PREFILL
 }
