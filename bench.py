@@ -910,7 +910,9 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="attn_1b", choices=sorted(gen.CONFIGS))
+    layer_set = {s.name: s for bits in (1, 2) for s in gen.LAYER_SET[bits]}
+    ap.add_argument("--workload", default="attn_1b", choices=sorted(gen.CONFIGS) + sorted(layer_set),
+                    help="a configuration, or one layer of the decoder-layer set (e.g. k_1b)")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-check", dest="check", action="store_false")
@@ -926,7 +928,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    shape = gen.CONFIGS[args.workload]
+    shape = gen.CONFIGS[args.workload] if args.workload in gen.CONFIGS else layer_set[args.workload]
     if args.factorize:
         run_factorize(args)
     elif args.profile_calls > 0:
