@@ -219,6 +219,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Let the next kernel in the stream be scheduled as this grid's CTAs exit
+  // (it waits for this grid's completion before it reads anything this grid
+  // writes).  Every CTA of this grid is resident once they have all passed
+  // here, so a dependent cannot keep one of them from starting; and two CTAs
+  // of this kernel never fit on one SM, so a dependent prefill CTA only takes
+  // an SM this grid has left.
+  pdl_launch_dependents();
   // Peers write into this CTA's receive buffer only after every CTA of the
   // cluster has initialised its barriers (the matching wait comes later).
   if constexpr (SPLIT) cluster_arrive_relaxed();
