@@ -894,10 +894,10 @@ def run_factorize(args):
         times.append(e0.elapsed_time(e1))
         errors.append(float(err.item()))
     steps = 20
-    # GEMMs of one pass: per factor G (k*k*inner), the right-hand product (rows*k*inner), Newton-Schulz 16 x 2 k^3,
-    # per ADMM step one (rows x k x k) product; the error product n*m*k
-    fl = 2.0 * (k * k * m + n * k * m + 32 * k ** 3 + steps * n * k * k) + 2.0 * (k * k * n + k * m * n + 32 * k ** 3 +
-                                                                                  steps * k * m * k) + 2.0 * n * m * k
+    # GEMMs of one pass: per factor G (k*k*inner), the right-hand product (rows*k*inner), the Cholesky factor and
+    # inverse (k^3 flops together), per ADMM step one (rows x k x k) product; the error product n*m*k
+    fl = 2.0 * (k * k * m + n * k * m + 0.5 * k ** 3 + steps * n * k * k) + 2.0 * (k * k * n + k * m * n + 0.5 * k ** 3 +
+                                                                                   steps * k * m * k) + 2.0 * n * m * k
     ms = statistics.median(times)
     print(json.dumps({"factorize": {"n": n, "m": m, "k": k, "bits_per_weight": k * (n + m) / (n * m),
                                     "start_ms": start_ms, "ms_per_pass": ms, "pass_ms": times,

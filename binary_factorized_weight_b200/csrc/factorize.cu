@@ -16,15 +16,17 @@
 //   err  = ||W - L R||_F / ||W||_F
 // Dense products are cuBLAS SGEMMs (fp32, no tensor-op math).  G is
 // symmetric positive definite with all eigenvalues in [rho, rho + lambda_max]
-// (rho is the mean eigenvalue of 2 R R^T), so its inverse comes from a fixed
-// number of Newton-Schulz steps X <- X (2I - G X) started at X = 2 / (lo + hi) I
-// with the Gershgorin bound hi (matrix products only).  SVID's rank-one
+// (rho is the mean eigenvalue of 2 R R^T, so its condition number is at most
+// k + 1), and its inverse comes from a Cholesky factorisation G = C C^T and
+// the inverse of the factor (cuSOLVER potrf / potri, about k^3 flops), formed
+// once per factor per pass so that every ADMM step is one GEMM.  SVID's rank-one
 // magnitude is the leading singular pair of |M| by power iteration from the
 // uniform vector (|M| is nonnegative: its leading pair is nonnegative and, for
 // the matrices met here, well separated).  Every reduction runs in a fixed
 // order (deterministic).
 #include <cublas_v2.h>
 #include <cuda_runtime.h>
+#include <cusolverDn.h>
 
 #include <mutex>
 
@@ -35,7 +37,6 @@ namespace dbf {
 namespace {
 
 constexpr int kT = 256;
-constexpr int kNewtonSteps = 16;
 constexpr int kPowerSteps = 30;
 constexpr int kMaxDev = 64;
 
@@ -49,6 +50,18 @@ cublasHandle_t handle_for(int device) {
     cublasHandle_t nh = nullptr;
     if (cublasCreate(&nh) != CUBLAS_STATUS_SUCCESS) return nullptr;
     cublasSetPointerMode(nh, CUBLAS_POINTER_MODE_HOST);
+    h[device] = nh;
+  }
+  return h[device];
+}
+
+cusolverDnHandle_t solver_for(int device) {
+  static cusolverDnHandle_t h[kMaxDev] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (h[device] == nullptr) {
+    cusolverDnHandle_t nh = nullptr;
+    if (cusolverDnCreate(&nh) != CUSOLVER_STATUS_SUCCESS) return nullptr;
     h[device] = nh;
   }
   return h[device];
@@ -88,9 +101,8 @@ __global__ void sumsq_kernel(const float* x, int64_t count, float* out) {
   if (threadIdx.x == 0) out[0] = s;
 }
 
-// G (k x k) += rho I with rho = trace(G) / k (G holds 2 R R^T), then
-// bounds: lo = rho, hi = max row sum of |G|; writes rho to scal[0] and the
-// Newton-Schulz start 2 / (lo + hi) to scal[1].  One CTA.
+// G (k x k) += rho I with rho = trace(G) / k (G holds 2 R R^T); writes rho
+// to scal[0].  One CTA.
 __global__ void regularize_kernel(float* G, int64_t k, float* scal) {
   __shared__ float red[kT / 32];
   __shared__ float s_rho;
@@ -101,39 +113,24 @@ __global__ void regularize_kernel(float* G, int64_t k, float* scal) {
   __syncthreads();
   const float rho = s_rho;
   for (int64_t i = threadIdx.x; i < k; i += kT) G[i * k + i] += rho;
-  __syncthreads();
-  float hi = 0.f;
-  for (int64_t i = threadIdx.x; i < k; i += kT) {
-    float rs = 0.f;
-    for (int64_t j = 0; j < k; ++j) rs += fabsf(G[i * k + j]);
-    hi = fmaxf(hi, rs);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = hi;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float h = 0.f;
-    for (int w = 0; w < kT / 32; ++w) h = fmaxf(h, red[w]);
-    scal[0] = rho;
-    scal[1] = 2.f / (rho + h);
-  }
+  if (threadIdx.x == 0) scal[0] = rho;
 }
 
-// X = c I (c = scal[1]), k x k.
-__global__ void scaled_identity_kernel(float* X, int64_t k, const float* scal) {
-  const float c = scal[1];
+// Gi (k x k) holds the inverse in its lower triangle (column-major, so the
+// upper triangle of the row-major array) after potri: mirror it into the other
+// half.  A failed factorisation (*info != 0, only possible for a non-finite
+// Gram) leaves NaN everywhere, so the pass's error is NaN and it is rejected.
+__global__ void mirror_inverse_kernel(float* Gi, int64_t k, const int* info) {
+  const bool bad = *info != 0;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < k * k;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    X[i] = (i / k == i % k) ? c : 0.f;
-}
-
-// Y = 2I - Y (k x k), in place.
-__global__ void two_minus_kernel(float* Y, int64_t k) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < k * k;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    Y[i] = ((i / k == i % k) ? 2.f : 0.f) - Y[i];
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / k, c = i % k;
+    if (bad) {
+      Gi[i] = __int_as_float(0x7fc00000);
+    } else if (r > c) {
+      Gi[i] = Gi[c * k + r];
+    }
+  }
 }
 
 // T = P + rho (Z - U)   (elementwise; P holds 2 W R^T or 2 L^T W)
@@ -307,17 +304,36 @@ FactWs fact_layout(char* base, int64_t n, int64_t m, int64_t k) {
   return w;
 }
 
-// Gi = G^-1 for G (k x k) symmetric positive definite with the bounds in scal.
-bool newton_inverse(cublasHandle_t h, const FactWs& w, int64_t k, int grid, cudaStream_t s) {
-  scaled_identity_kernel<<<grid, kT, 0, s>>>(w.Gi, k, w.scal);
-  for (int it = 0; it < kNewtonSteps; ++it) {
-    if (!gemm(h, false, false, k, k, k, 1.f, w.G, w.Gi, 0.f, w.Y)) return false;  // Y = G X
-    two_minus_kernel<<<grid, kT, 0, s>>>(w.Y, k);                                  // Y = 2I - G X
-    if (!gemm(h, false, false, k, k, k, 1.f, w.Gi, w.Y, 0.f, w.X2)) return false;  // X (2I - G X)
-    if (cudaMemcpyAsync(w.Gi, w.X2, static_cast<size_t>(k * k) * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return false;
+// Gi = G^-1 for G (k x k) symmetric positive definite: Cholesky factor of a
+// copy, inverse from the factor, mirrored to a full matrix.  The solver's
+// scratch is the k x k pair Y, X2 when its request fits there (large k), else
+// a stream-ordered allocation freed on the same stream; its status word sits
+// in the scalar area.
+dbf_status cholesky_inverse(cusolverDnHandle_t sh, const FactWs& w, int64_t k, int grid, cudaStream_t s) {
+  const int kk = static_cast<int>(k);
+  const size_t cap = static_cast<size_t>(w.X2 - w.Y) + static_cast<size_t>(k * k);  // floats in Y..X2
+  int lw_f = 0, lw_i = 0;
+  if (cudaMemcpyAsync(w.Gi, w.G, static_cast<size_t>(k * k) * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return DBF_ERR_CUDA;
+  if (cusolverDnSpotrf_bufferSize(sh, CUBLAS_FILL_MODE_LOWER, kk, w.Gi, kk, &lw_f) != CUSOLVER_STATUS_SUCCESS ||
+      cusolverDnSpotri_bufferSize(sh, CUBLAS_FILL_MODE_LOWER, kk, w.Gi, kk, &lw_i) != CUSOLVER_STATUS_SUCCESS)
+    return DBF_ERR_CUDA;
+  const int lw = lw_f > lw_i ? lw_f : lw_i;
+  if (lw < 0) return DBF_ERR_CUDA;
+  float* scratch = w.Y;
+  void* own = nullptr;
+  if (static_cast<size_t>(lw) > cap) {
+    if (cudaMallocAsync(&own, static_cast<size_t>(lw) * 4, s) != cudaSuccess) return DBF_ERR_CUDA;
+    scratch = static_cast<float*>(own);
   }
-  return true;
+  int* info = reinterpret_cast<int*>(w.scal + 16);
+  const bool ok =
+      cusolverDnSpotrf(sh, CUBLAS_FILL_MODE_LOWER, kk, w.Gi, kk, scratch, lw, info) == CUSOLVER_STATUS_SUCCESS &&
+      cusolverDnSpotri(sh, CUBLAS_FILL_MODE_LOWER, kk, w.Gi, kk, scratch, lw, info) == CUSOLVER_STATUS_SUCCESS;
+  if (own && cudaFreeAsync(own, s) != cudaSuccess) return DBF_ERR_CUDA;
+  if (!ok) return DBF_ERR_CUDA;
+  mirror_inverse_kernel<<<grid, kT, 0, s>>>(w.Gi, k, info);
+  return cudaGetLastError() == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
 // One ADMM solve of a factor F (rows x cols, in/out, SVID form) with P = the
@@ -419,23 +435,27 @@ dbf_status dbf_factorize_pass(const float* W, int64_t n, int64_t m, int64_t k, f
   st = current_device(&dev);
   if (st != DBF_OK) return st;
   cublasHandle_t h = handle_for(dev.device);
-  if (!h) return DBF_ERR_CUDA;
+  cusolverDnHandle_t sh = solver_for(dev.device);
+  if (!h || !sh) return DBF_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_handle);
-  if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return DBF_ERR_CUDA;
+  if (cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS || cusolverDnSetStream(sh, s) != CUSOLVER_STATUS_SUCCESS)
+    return DBF_ERR_CUDA;
   const FactWs w = fact_layout(static_cast<char*>(workspace), n, m, k);
   const int grid = 4 * dev.num_sms;
 
   // left factor, R fixed
   if (!gemm(h, false, true, k, k, m, 2.f, R, R, 0.f, w.G)) return DBF_ERR_CUDA;  // 2 R R^T
   regularize_kernel<<<1, kT, 0, s>>>(w.G, k, w.scal);
-  if (!newton_inverse(h, w, k, grid, s)) return DBF_ERR_CUDA;
+  st = cholesky_inverse(sh, w, k, grid, s);
+  if (st != DBF_OK) return st;
   if (!gemm(h, false, true, n, k, m, 2.f, W, R, 0.f, w.P)) return DBF_ERR_CUDA;  // 2 W R^T
   st = admm_factor(h, w, L, n, k, true, admm_steps, grid, s);
   if (st != DBF_OK) return st;
   // right factor, L fixed
   if (!gemm(h, true, false, k, k, n, 2.f, L, L, 0.f, w.G)) return DBF_ERR_CUDA;  // 2 L^T L
   regularize_kernel<<<1, kT, 0, s>>>(w.G, k, w.scal);
-  if (!newton_inverse(h, w, k, grid, s)) return DBF_ERR_CUDA;
+  st = cholesky_inverse(sh, w, k, grid, s);
+  if (st != DBF_OK) return st;
   if (!gemm(h, true, false, k, m, n, 2.f, L, W, 0.f, w.P)) return DBF_ERR_CUDA;  // 2 L^T W
   st = admm_factor(h, w, R, k, m, false, admm_steps, grid, s);
   if (st != DBF_OK) return st;

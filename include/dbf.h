@@ -409,9 +409,12 @@ DBF_API dbf_status dbf_bqq_forward(const uint16_t* x, const uint32_t* packedY, c
  *   workspace: dbf_factorize_workspace_bytes(n, m, k) bytes of device memory.
  *   Shape: n, m <= 65536, k <= 16384, n*m and k*max(n, m) <= 2^31.
  *   Arithmetic: fp32 (cuBLAS SGEMM for the dense products, no tensor-op math);
- *   G^-1 by 16 Newton-Schulz steps (G's eigenvalues lie in [rho, rho +
- *   lambda_max(2 R R^T)], rho their mean); SVID's magnitudes by 30 power
- *   steps on |M|.  Deterministic.
+ *   G^-1 from a Cholesky factorisation (cuSOLVER potrf / potri; G's
+ *   eigenvalues lie in [rho, rho + lambda_max(2 R R^T)], rho their mean, so
+ *   it is well conditioned); SVID's magnitudes by 30 power steps on |M|.
+ *   Deterministic.  The solver's scratch lives in the workspace when it fits
+ *   in 2 k^2 floats, else it is taken from and returned to the stream-ordered
+ *   allocator of the current device within the call (small k only).
  * dbf_svid: the leading singular pair of |M| (rows x cols, fp32): unit vectors
  *   u (rows) and v (cols) and sigma (one fp32), all device memory (scratch:
  *   dbf_svid_workspace_bytes(rows, cols) bytes of device workspace), so that
