@@ -92,12 +92,25 @@ __device__ float block_sum(float v, float* red) {
   return s;
 }
 
-// out[0] = sum of squares of x (count elements), one CTA.
-__global__ void sumsq_kernel(const float* x, int64_t count, float* out) {
+// Sum of squares of x (count elements) in two launches with a fixed order:
+// CTA c sums a strided share (fp64 per thread) into part[c], then one CTA adds
+// the kSumCtas parts.
+constexpr int kSumCtas = 256;
+
+__global__ void sumsq_part_kernel(const float* x, int64_t count, float* part) {
   __shared__ float red[kT / 32];
   double acc = 0.0;  // long sums: accumulate in fp64 per thread
-  for (int64_t i = threadIdx.x; i < count; i += kT) acc += static_cast<double>(x[i]) * x[i];
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(kT) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(kSumCtas) * kT)
+    acc += static_cast<double>(x[i]) * x[i];
   const float s = block_sum(static_cast<float>(acc), red);
+  if (threadIdx.x == 0) part[blockIdx.x] = s;
+}
+
+__global__ void sum_final_kernel(const float* part, float* out) {
+  __shared__ float red[kT / 32];
+  static_assert(kSumCtas == kT, "one part per thread");
+  const float s = block_sum(part[threadIdx.x], red);
   if (threadIdx.x == 0) out[0] = s;
 }
 
@@ -163,10 +176,18 @@ __global__ void fill_kernel(float* u, int64_t count, float c) {
     u[i] = c;
 }
 
-// part[c][j] = sum over rows i of chunk c of |M[i][j]| u[i]   (rows x cols
-// row-major; a thread per column and chunk, the chunk's rows in order)
+// part[c][j] = sum over rows i of chunk c of |M[i][j]| u[i] / ||u||   (rows x
+// cols row-major; a thread per column and chunk, the chunk's rows in order).
+// Every CTA forms ||u|| itself in the same fixed order (no separate
+// normalisation launch for u).
 constexpr int kRowChunks = 32;
 __global__ void abs_gemv_t_part_kernel(const float* M, const float* u, int64_t rows, int64_t cols, float* part) {
+  __shared__ float red[kT / 32];
+  float q = 0.f;
+  for (int64_t i = threadIdx.x; i < rows; i += kT) q = fmaf(u[i], u[i], q);
+  q = block_sum(q, red);
+  const float nrm = sqrtf(q);
+  const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
   const int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t c = blockIdx.y;
   if (j >= cols) return;
@@ -174,7 +195,7 @@ __global__ void abs_gemv_t_part_kernel(const float* M, const float* u, int64_t r
   const int64_t i1 = (c + 1) * per < rows ? (c + 1) * per : rows;
   float s = 0.f;
   for (int64_t i = c * per; i < i1; ++i) s = fmaf(fabsf(M[i * cols + j]), u[i], s);
-  part[c * cols + j] = s;
+  part[c * cols + j] = s * inv;
 }
 
 // v[j] = sum of the chunks' parts in chunk order
@@ -186,8 +207,16 @@ __global__ void sum_parts_kernel(const float* part, int64_t cols, float* v) {
   v[j] = s;
 }
 
-// u[i] = sum_j |M[i][j]| v[j]   (a warp per row, lanes over the row, fixed-order tree)
+// u[i] = sum_j |M[i][j]| v[j] / ||v||   (a warp per row, lanes over the row,
+// fixed-order tree).  Every CTA forms ||v|| itself in the same fixed order, so
+// the power step needs no separate normalisation launch for v.
 __global__ void abs_gemv_kernel(const float* M, const float* v, int64_t rows, int64_t cols, float* u) {
+  __shared__ float red[kT / 32];
+  float q = 0.f;
+  for (int64_t j = threadIdx.x; j < cols; j += kT) q = fmaf(v[j], v[j], q);
+  q = block_sum(q, red);
+  const float nrm = sqrtf(q);
+  const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
   const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (i >= rows) return;
@@ -195,7 +224,7 @@ __global__ void abs_gemv_kernel(const float* M, const float* v, int64_t rows, in
   for (int64_t j = lane; j < cols; j += 32) s = fmaf(fabsf(M[i * cols + j]), v[j], s);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) u[i] = s;
+  if (lane == 0) u[i] = s * inv;
 }
 
 // x /= ||x|| (one CTA); if nrm_out, *nrm_out = ||x|| before the division.
@@ -237,15 +266,17 @@ __global__ void ratio_sqrt_kernel(const float* num, const float* den, float* out
 // part: kRowChunks * cols floats of scratch.
 dbf_status svid_pair(const float* M, int64_t rows, int64_t cols, float* u, float* v, float* sigma, float* part,
                      int grid, cudaStream_t s) {
-  fill_kernel<<<grid, kT, 0, s>>>(u, rows, 1.f / sqrtf(static_cast<float>(rows)));
+  fill_kernel<<<grid, kT, 0, s>>>(u, rows, 1.f);
   const unsigned cblocks = static_cast<unsigned>((cols + kT - 1) / kT);
   for (int it = 0; it < kPowerSteps; ++it) {
     abs_gemv_t_part_kernel<<<dim3(cblocks, kRowChunks), kT, 0, s>>>(M, u, rows, cols, part);
     sum_parts_kernel<<<cblocks, kT, 0, s>>>(part, cols, v);
-    normalize_kernel<<<1, kT, 0, s>>>(v, cols, nullptr);
     abs_gemv_kernel<<<static_cast<unsigned>((rows * 32 + kT - 1) / kT), kT, 0, s>>>(M, v, rows, cols, u);
-    normalize_kernel<<<1, kT, 0, s>>>(u, rows, sigma);
   }
+  // u = |M| v / ||v|| of the last step: sigma = ||u||; both vectors to unit
+  // length (inside the loop each product normalises its input vector itself)
+  normalize_kernel<<<1, kT, 0, s>>>(v, cols, nullptr);
+  normalize_kernel<<<1, kT, 0, s>>>(u, rows, sigma);
   return cudaGetLastError() == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
 
@@ -366,8 +397,10 @@ dbf_status rel_error(cublasHandle_t h, const FactWs& w, const float* W, const fl
                      int64_t m, int64_t k, float* err, int grid, cudaStream_t s) {
   if (!gemm(h, false, false, n, m, k, 1.f, L, R, 0.f, w.E)) return DBF_ERR_CUDA;
   residual_kernel<<<grid, kT, 0, s>>>(W, w.E, n * m);
-  sumsq_kernel<<<1, kT, 0, s>>>(w.E, n * m, w.scal + 4);
-  sumsq_kernel<<<1, kT, 0, s>>>(W, n * m, w.scal + 5);
+  sumsq_part_kernel<<<kSumCtas, kT, 0, s>>>(w.E, n * m, w.part);
+  sum_final_kernel<<<1, kT, 0, s>>>(w.part, w.scal + 4);
+  sumsq_part_kernel<<<kSumCtas, kT, 0, s>>>(W, n * m, w.part);
+  sum_final_kernel<<<1, kT, 0, s>>>(w.part, w.scal + 5);
   ratio_sqrt_kernel<<<1, 1, 0, s>>>(w.scal + 4, w.scal + 5, err);
   return cudaGetLastError() == cudaSuccess ? DBF_OK : DBF_ERR_CUDA;
 }
