@@ -208,23 +208,26 @@ __global__ void sum_parts_kernel(const float* part, int64_t cols, float* v) {
 }
 
 // u[i] = sum_j |M[i][j]| v[j] / ||v||   (a warp per row, lanes over the row,
-// fixed-order tree).  Every CTA forms ||v|| itself in the same fixed order, so
-// the power step needs no separate normalisation launch for v.
+// fixed-order tree).  Each warp reads all of v for its row, so it forms ||v||
+// in the same loop, in the same order in every warp: the power step needs no
+// separate normalisation launch for v.
 __global__ void abs_gemv_kernel(const float* M, const float* v, int64_t rows, int64_t cols, float* u) {
-  __shared__ float red[kT / 32];
-  float q = 0.f;
-  for (int64_t j = threadIdx.x; j < cols; j += kT) q = fmaf(v[j], v[j], q);
-  q = block_sum(q, red);
-  const float nrm = sqrtf(q);
-  const float inv = nrm > 0.f ? 1.f / nrm : 0.f;
   const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (i >= rows) return;
-  float s = 0.f;
-  for (int64_t j = lane; j < cols; j += 32) s = fmaf(fabsf(M[i * cols + j]), v[j], s);
+  float s = 0.f, q = 0.f;
+  for (int64_t j = lane; j < cols; j += 32) {
+    const float vj = v[j];
+    s = fmaf(fabsf(M[i * cols + j]), vj, s);
+    q = fmaf(vj, vj, q);
+  }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) u[i] = s * inv;
+  for (int off = 16; off > 0; off >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, off);
+    q += __shfl_xor_sync(0xffffffffu, q, off);
+  }
+  const float nrm = sqrtf(q);
+  if (lane == 0) u[i] = nrm > 0.f ? s * (1.f / nrm) : 0.f;
 }
 
 // x /= ||x|| (one CTA); if nrm_out, *nrm_out = ||x|| before the division.
