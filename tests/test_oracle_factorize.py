@@ -12,7 +12,13 @@ equations, so the reference is pinned by what the mathematics fixes:
   * the error falls as k grows (the analogue of the pages' error-vs-size
     curves), and at every k it is below 1 (the zero matrix);
   * the returned factors reconstruct, through the pinned C oracle's dense
-    weight, exactly what the factorisation reports.
+    weight, exactly what the factorisation reports;
+  * a converged ADMM solve sits at a fixed point of scaled ADMM: L = Z (the
+    dual update stops) and Z = SVID(Z - grad f(Z) / rho) for the least-squares
+    term f(L) = ||W - L R||_F^2 (the L step's stationarity fixes the scaled dual
+    at U = -grad f(Z) / rho, and the Z step then projects Z + U);
+  * a pass that would raise the error is not kept (on a seeded case where one
+    does).
 """
 import numpy as np
 import pytest
@@ -84,3 +90,35 @@ def test_factors_reconstruct_through_the_dense_oracle(oracle_mod):
     Wd = oracle_mod.dense_weight(f["A"], f["B"], f["a"], f["mid"], f["b"])
     assert np.allclose(Wd, F.reconstruct(f), rtol=1e-12, atol=1e-12)
     assert np.linalg.norm(W - Wd) / np.linalg.norm(W) == pytest.approx(f["errors"][-1], rel=1e-9)
+
+
+@pytest.mark.parametrize("seed", [300, 302])
+def test_converged_admm_is_a_projected_gradient_fixed_point(seed):
+    rng = np.random.default_rng(seed)
+    n, m, k = 12, 10, 3
+    W = rng.standard_normal((n, m))
+    R = F.svid_matrix(rng.standard_normal((k, m)))
+    Z0 = F.svid_matrix(rng.standard_normal((n, k)))
+    rho = 2.0 * float(np.sum(R * R)) / k
+    Z = F.admm_left(W, R, Z0, rho, 400)
+    Z_next = F.admm_left(W, R, Z0, rho, 401)
+    # these seeded cases converge (ADMM on a nonconvex set need not)
+    assert np.linalg.norm(Z_next - Z) <= 1e-12 * np.linalg.norm(Z)
+    grad = -2.0 * (W - Z @ R) @ R.T  # gradient of ||W - L R||_F^2 at L = Z
+    assert np.linalg.norm(F.svid_matrix(Z - grad / rho) - Z) <= 1e-10 * np.linalg.norm(Z)
+
+
+def test_a_pass_that_raises_the_error_is_not_kept():
+    W = np.random.default_rng(202).standard_normal((16, 48))
+    Om = gen.projection_signs(np.random.default_rng(2), 48, 8)
+    L, R = F.start_factors(W, Om)
+    free = [F.relative_error(W, L, R)]
+    for _ in range(8):
+        L, R = F.alternating_pass(W, L, R, 20)
+        free.append(F.relative_error(W, L, R))
+    assert any(free[i + 1] > free[i] for i in range(8)), "the case must contain a rising pass"
+    e = F.factorize(W, Om, passes=8, admm_steps=20)["errors"]
+    assert all(e[i + 1] <= e[i] for i in range(8))
+    first_rise = next(i for i in range(8) if free[i + 1] > free[i])
+    assert e[:first_rise + 1] == pytest.approx(free[:first_rise + 1], rel=1e-12)
+    assert e[first_rise + 1] == e[first_rise]
