@@ -749,13 +749,18 @@ def run_sweep(args):
         gbs = wl.bytes / (us * 1e-6) / 1e9
         tf = layer_flops(shape.n, shape.k, shape.m_in, batch) / (us * 1e-6) / 1e12
         dense_us = dense_fp16_us(torch, shape, batch, device)
+        dense_bytes = 2 * shape.n * shape.m_in + 2 * batch * (shape.n + shape.m_in)  # fp16 W, x and y once
+        dense_floor_us = dense_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6
         row = {"layer": shape.name, "n": shape.n, "k": shape.k, "m_in": shape.m_in, "batch": batch,
                "bpw": shape.k * (shape.n + shape.m_in) / (shape.n * shape.m_in), "us": us,
                "us_p10": sorted(times)[0], "us_p90": sorted(times)[-1], "tokens_per_s": batch / (us * 1e-6),
                "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": tf,
                "tensor_frac": tf / peaks["bf16_tflops"], "copies": wl.copies, "path": wl.path,
                "context_torch_fp16_dense_us": dense_us,
-               "speedup_vs_dense_fp16": dense_us / us}
+               "context_dense_hbm_frac": dense_bytes / (dense_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+               "speedup_vs_dense_fp16": dense_us / us,
+               "dense_fp16_hbm_floor_us": dense_floor_us,
+               "speedup_vs_dense_hbm_floor": dense_floor_us / us}
         rows.append(row)
         print(json.dumps(row), flush=True)
         del g, wl
