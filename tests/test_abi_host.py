@@ -215,3 +215,112 @@ def test_forward_transposed_validation(lib):
     assert call(k=96) == SHAPE
     assert call(dx=MIS) == MISALIGNED
     assert call(ws_bytes=255) == WORKSPACE
+
+
+def no_device():
+    import torch
+
+    return not torch.cuda.is_available()
+
+
+def test_factorize_workspace_bytes(lib):
+    f = lib.dbf_factorize_workspace_bytes
+    assert f(0, 4, 4) == 0 and f(4, 0, 4) == 0 and f(4, 4, 0) == 0
+    assert f(65537, 4, 4) == 0 and f(4, 65537, 4) == 0 and f(4, 4, 16385) == 0
+    assert f(65536, 65536, 1) == 0          # n * m above 2^31
+    assert f(65536, 64, 16384) > 0          # the largest factor: 2^30 elements
+    n, m, k = 4096, 4096, 2048
+    # at least: W - L R (n x m), six factor-sized buffers, the Gram matrix and its inverse with the
+    # solver's two k x k slots, all fp32
+    assert f(n, m, k) >= 4 * (n * m + 6 * max(n, m) * k + 4 * k * k)
+    assert f(n, m, k) % 256 == 0
+    assert f(n, m, 2 * k) > f(n, m, k)
+
+
+def test_svid_workspace_bytes(lib):
+    assert lib.dbf_svid_workspace_bytes(4096, 2048) == 32 * 2048 * 4  # 32 row chunks of fp32 column sums
+    assert lib.dbf_svid_workspace_bytes(1, 1) == 32 * 4
+    assert lib.dbf_svid_workspace_bytes(0, 5) == 0 and lib.dbf_svid_workspace_bytes(5, 0) == 0
+
+
+def test_svid_validation(lib):
+    def call(M=P, rows=64, cols=32, u=P, v=P, sigma=P, ws=P, ws_bytes=1 << 20):
+        return lib.dbf_svid(M, rows, cols, u, v, sigma, ws, ws_bytes, None)
+
+    for bad in ("M", "u", "v", "sigma", "ws"):
+        assert call(**{bad: None}) == INVALID, bad
+    assert call(rows=0) == INVALID and call(cols=-1) == INVALID
+    assert call(rows=1 << 16, cols=(1 << 15) + 1) == SHAPE
+    for bad in ("M", "u", "v", "sigma", "ws"):
+        assert call(**{bad: MIS}) == MISALIGNED, bad
+    assert call(ws_bytes=32 * 32 * 4 - 1) == WORKSPACE
+    if no_device():
+        assert call(ws_bytes=32 * 32 * 4) in (CUDA_ERR, 7)
+
+
+def test_factorize_validation(lib):
+    ws_ok = lib.dbf_factorize_workspace_bytes(200, 256, 64)
+
+    def pass_(W=P, n=200, m=256, k=64, L=P, R=P, steps=20, err=P, ws=P, ws_bytes=ws_ok):
+        return lib.dbf_factorize_pass(W, n, m, k, L, R, steps, err, ws, ws_bytes, None)
+
+    def start(W=P, Om=P, n=200, m=256, k=64, L=P, R=P, err=P, ws=P, ws_bytes=ws_ok):
+        return lib.dbf_factorize_start(W, Om, n, m, k, L, R, err, ws, ws_bytes, None)
+
+    def finish(L=P, R=P, n=200, m=256, k=64, pA=P, pB=P, a=P, mid=P, b=P, ws=P, ws_bytes=ws_ok):
+        return lib.dbf_factorize_finish(L, R, n, m, k, pA, pB, a, mid, b, ws, ws_bytes, None)
+
+    for call, ptrs in ((pass_, ("W", "L", "R", "err", "ws")), (start, ("W", "Om", "L", "R", "err", "ws")),
+                       (finish, ("L", "R", "pA", "pB", "a", "mid", "b", "ws"))):
+        for name in ptrs:
+            assert call(**{name: None}) == INVALID, (call.__name__, name)
+            assert call(**{name: MIS}) == MISALIGNED, (call.__name__, name)
+        assert call(n=0) == INVALID and call(k=0) == INVALID
+        assert call(n=65537) == SHAPE and call(k=16385) == SHAPE and call(n=65536, m=65536, k=1) == SHAPE
+        assert call(ws_bytes=ws_ok - 1) == WORKSPACE
+        if no_device():
+            assert call() in (CUDA_ERR, 7), call.__name__
+    assert pass_(steps=0) == INVALID and pass_(steps=1001) == INVALID
+
+
+def test_bqq_sizes(lib):
+    # (n, k, p, m_in): p terms of k middle rows each, p * k and m_in multiples of 64
+    assert lib.dbf_bqq_prepared_bytes(256, 32, 2, 256) > 0
+    assert lib.dbf_bqq_prepared_bytes(256, 32, 1, 256) == 0      # p * k = 32 is not a multiple of 64
+    assert lib.dbf_bqq_prepared_bytes(256, 64, 1, 100) == 0      # m_in not a multiple of 64
+    assert lib.dbf_bqq_prepared_bytes(256, 64, 4097, 256) == 0   # more than 4096 terms
+    assert lib.dbf_bqq_prepared_bytes(0, 64, 1, 256) == 0
+    # the DBF forward's workspace for the k p middle rows, then the fp32 sign-product term (batch x n)
+    for n, k, p, m_in, batch in ((256, 32, 2, 256, 4), (4096, 256, 8, 4096, 2048), (100, 64, 3, 64, 1)):
+        assert lib.dbf_bqq_workspace_bytes(n, k, p, m_in, batch) == \
+            lib.dbf_forward_workspace_bytes(n, k * p, m_in, batch) + (batch * n * 4 + 255) // 256 * 256
+    assert lib.dbf_bqq_workspace_bytes(256, 32, 2, 256, 0) == 0
+
+
+def test_bqq_validation(lib):
+    prep_ok = lib.dbf_bqq_prepared_bytes(256, 32, 2, 256)
+    ws_ok = lib.dbf_bqq_workspace_bytes(256, 32, 2, 256, 4)
+
+    def prepare(Y=P, Z=P, r=P, s=P, t=P, u=P, n=256, k=32, p=2, m_in=256, prep=P, prep_bytes=prep_ok):
+        return lib.dbf_bqq_prepare(Y, Z, r, s, t, u, n, k, p, m_in, prep, prep_bytes, None)
+
+    def forward(x=P, Y=P, Z=P, prep=P, n=256, k=32, p=2, m_in=256, batch=4, y=P, y_t=1, ws=P, ws_bytes=ws_ok,
+                flags=0):
+        return lib.dbf_bqq_forward(x, Y, Z, prep, n, k, p, m_in, batch, y, y_t, ws, ws_bytes, flags, None)
+
+    for name in ("Y", "Z", "r", "s", "t", "u", "prep"):
+        assert prepare(**{name: None}) == INVALID, name
+    assert prepare(k=48) == SHAPE and prepare(m_in=100) == SHAPE and prepare(n=0) == INVALID
+    for name in ("Y", "Z", "prep"):
+        assert prepare(**{name: MIS}) == MISALIGNED, name
+    assert prepare(prep_bytes=prep_ok - 1) == WORKSPACE
+    for name in ("x", "Y", "Z", "prep", "y"):
+        assert forward(**{name: None}) == INVALID, name
+    assert forward(k=48) == SHAPE and forward(batch=0) == INVALID and forward(y_t=7) == INVALID
+    assert forward(flags=1 << 9) == INVALID
+    for name in ("x", "Y", "Z", "prep", "y"):
+        assert forward(**{name: MIS}) == MISALIGNED, name
+    assert forward(ws=None) == WORKSPACE and forward(ws=MIS) == WORKSPACE and forward(ws_bytes=ws_ok - 1) == WORKSPACE
+    if no_device():
+        assert prepare() in (CUDA_ERR, 7)
+        assert forward() in (CUDA_ERR, 7)
